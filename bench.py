@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Decode-step throughput of the BasisKV hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one decode step of one attention layer for every sequence of the
+batch: append (latent + residual + page summary), route (page scores + top-k),
+decode_attn (exact attention on the routed pages), out_proj (fused factor).
+The metric is decode tokens/s per layer (batch / step time).  Each C-ABI call
+is captured once into its own CUDA graph; a timed step replays the four graphs
+with CUDA events between them on the launching stream.  L2 is flushed between
+steps by reading a 256 MiB buffer (outside the events).
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica on its own sequences (weak scaling; the path has no exchange step).
+``--impl reference`` times the fp64 CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from long_context_decode_basiskv_b200.workloads import WORKLOADS, make_case  # noqa: E402
+
+METRIC = "decode tokens/s per layer on 1 B200; route+attn HBM GB/s vs ~8 TB/s roofline"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNELS_PER_STEP = 7  # append 1, route 2 (score, select), decode_attn 3 (union, attn, combine), out_proj 1
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama3_8b_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--oracle-seqs", type=int, default=2, help="sequences in the CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, sampled from a thread)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # noqa: BLE001
+            self.err = repr(exc)
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                try:
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append(mhz)
+                self.reasons |= int(rs)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must move)
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(eng):
+    case, cfg = eng.case, eng.cfg
+    wl = case.wl
+    es = 2 if wl.dtype == "bf16" else 4
+    B, Hq, Hkv, d, r, s, P, k = (wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.rank_v,
+                                 wl.rank_k, wl.page_size, wl.top_k)
+    G = Hq // Hkv
+    pages = [-(-L // P) for L in case.lengths]
+    sel = eng.sel.cpu().numpy()
+    cnt = eng.sel_cnt.cpu().numpy()
+    union = 0
+    for b in range(B):
+        for g in range(Hkv):
+            u = set()
+            for h in range(g * G, (g + 1) * G):
+                u.update(sel[b, h, :cnt[b, h]].tolist())
+            union += len(u)
+    q_bytes = B * Hq * d * es
+    sel_bytes = B * Hq * (k + 2) * 4
+    route = sum(pages) * Hkv * d * 4 + 2 * sum(pages) * Hq * 4 + q_bytes + sel_bytes
+    decode = union * P * (d + r) * es + q_bytes + sel_bytes + B * Hq * r * 4
+    out = Hq * r * wl.hidden * es + B * Hq * r * 4 + B * wl.hidden * 4
+    append = B * Hkv * ((2 * d * r + d * s) * es + 2 * d * es + P * (r + s) * es + d * 4)
+    return {"append": append, "route": route, "decode_attn": decode, "out_proj": out,
+            "union_pages": union}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(kernel_file: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, "long_context_decode_basiskv_b200", "csrc", kernel_file)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if rec.get("source_sha256") != sha:
+            return None
+        return rec
+    except Exception:  # noqa: BLE001
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def oracle_sample(case, nseq: int, repeats: int = 1):
+    """Time the oracle's decode step (append .. out-projection) on `nseq` sequences.
+
+    The prefill of each sequence's oracle cache is untimed.  A repeat re-runs
+    the same decode step (the cache length is reset before the append).
+    Returns (seconds per decode step list, description).
+    """
+    from threadpoolctl import threadpool_limits
+
+    from oracle import basiskv_oracle as O
+
+    wl = case.wl
+    storage = "f32" if wl.dtype == "f32" else "bf16"
+
+    def f64(t):
+        return t.detach().to("cpu").to(torch.float64).numpy()
+
+    A, P, E = f64(case.A), f64(case.P), f64(case.E)
+    times = []
+    with threadpool_limits(1):
+        G = O.fuse_out_factor(f64(case.Bf), f64(case.W_O), wl.num_q_heads, storage)
+        for b in range(min(nseq, wl.batch)):
+            K, V = f64(case.keys[b]), f64(case.values[b])
+            L = K.shape[0]
+            cache = O.prefill(K[:-1], V[:-1], A, P, E, wl.page_size, storage, capacity=L)
+            q = f64(case.q[b])
+            for _ in range(repeats):
+                cache.length = L - 1
+                t0 = time.perf_counter()
+                O.decode_step(cache, K[-1], V[-1], q, A, P, E, G, wl.top_k)
+                times.append(time.perf_counter() - t0)
+    desc = (f"fp64 numpy oracle, 1 thread: decode step (append, summary, route, attention, "
+            f"out-projection) of {min(nseq, wl.batch)} of the {wl.batch} sequences x {repeats}, "
+            f"prefill untimed")
+    return times, desc
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    from long_context_decode_basiskv_b200.engine import DecodeEngine
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    wl = WORKLOADS[args.workload]
+    if world > 1:
+        wl = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)   # different sequences per replica
+    case = make_case(wl, dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        eng = DecodeEngine(case, device=dev)
+        eng.step()
+    torch.cuda.synchronize()
+    if int(eng.err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(eng.err.item())}")
+    nbytes = algorithmic_bytes(eng)
+
+    # one CUDA graph per C-ABI call
+    graphs = {}
+    for name, fn in [("append", eng.append), ("route", eng.route), ("decode_attn", eng.decode_attn),
+                     ("out_proj", eng.out_proj)]:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        graphs[name] = g
+    torch.cuda.synchronize()
+    order = ["append", "route", "decode_attn", "out_proj"]
+    flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
+    sink = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def run_steps(n, record):
+        evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                torch.sum(flush, dim=0, out=sink)
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
+                if record:
+                    e[0].record(stream)
+                for i, name in enumerate(order):
+                    graphs[name].replay()
+                    if record:
+                        e[i + 1].record(stream)
+                if record:
+                    evs.append(e)
+        return evs
+
+    run_steps(args.warmup, False)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        evs = run_steps(args.steps, True)
+        torch.cuda.synchronize()
+    barrier(world)
+    per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, name in enumerate(order)}
+    step_ms = [ev[0].elapsed_time(ev[4]) for ev in evs]
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    ms_per_step = total_ms / args.steps
+    value = world * wl.batch * args.steps / (total_ms / 1e3)
+
+    mean = {k: sum(v) / len(v) for k, v in per.items()}
+    peak, peak_kind = measured_peak()
+    attn_gbs = nbytes["decode_attn"] / (mean["decode_attn"] * 1e-3) / 1e9
+    ra_gbs = (nbytes["route"] + nbytes["decode_attn"]) / ((mean["route"] + mean["decode_attn"]) * 1e-3) / 1e9
+    traffic_rec = profiled_traffic("decode_attn.cu")
+    roofline = {
+        "kernel": "basiskv_decode_attn (union + attn + combine launches)",
+        "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
+        "frac": round(attn_gbs / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+        "algorithmic_bytes": nbytes["decode_attn"],
+        "traffic": traffic_rec["dram_bytes_per_launch"] if traffic_rec else None,
+    }
+
+    # end to end through the public API: pinned host inputs -> step -> host output
+    e2e = None
+    if not args.no_e2e:
+        hq = eng.q.cpu().pin_memory()
+        hk = eng.k_new.cpu().pin_memory()
+        hv = eng.v_new.cpu().pin_memory()
+        hy = torch.empty(eng.y.shape, dtype=eng.y.dtype).pin_memory()
+        bi = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+        bo = hy.numel() * hy.element_size()
+
+        def e2e_steps(n, record):
+            out = []
+            with torch.cuda.stream(stream):
+                for _ in range(n):
+                    torch.sum(flush, dim=0, out=sink)
+                    if record:
+                        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        a.record(stream)
+                    eng.q.copy_(hq, non_blocking=True)
+                    eng.k_new.copy_(hk, non_blocking=True)
+                    eng.v_new.copy_(hv, non_blocking=True)
+                    eng.step()
+                    hy.copy_(eng.y, non_blocking=True)
+                    if record:
+                        b_.record(stream)
+                        out.append((a, b_))
+            return out
+
+        e2e_steps(max(3, args.warmup), False)
+        torch.cuda.synchronize()
+        barrier(world)
+        pairs = e2e_steps(args.steps, True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in pairs), world, dev)
+        e2e = {"value": round(world * wl.batch * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+               "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        times, desc = oracle_sample(case, args.oracle_seqs)
+        cpu = {"value": round(len(times) / sum(times), 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": desc, "seconds": round(sum(times), 3)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic (seeded generator)",
+            "config": {"workload": wl.name, "batch": wl.batch, "context": wl.context if not wl.ragged else list(wl.ragged),
+                       "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                       "page_size": wl.page_size, "rank_v": wl.rank_v, "rank_k": wl.rank_k,
+                       "top_k": wl.top_k, "hidden": wl.hidden, "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (read of a 256 MiB buffer)",
+                       "timing": "one CUDA graph per C-ABI call, CUDA events between them"},
+            "kernels_us": {k: round(v * 1e3, 2) for k, v in mean.items()},
+            "algorithmic_bytes": nbytes,
+            "route_attn_gbs": round(ra_gbs, 1),
+            "route_attn_frac_of_8tbs": round(ra_gbs / 8000.0, 4),
+            "route_attn_frac_of_measured": round(ra_gbs / peak, 4),
+            "roofline": roofline,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    case = make_case(wl, "cpu")
+    times, desc = oracle_sample(case, 1, repeats=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    value = len(timed) / sum(timed)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * sum(timed) / len(timed), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
+        "config": {"workload": wl.name, "batch": wl.batch, "sample": "one sequence per step"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

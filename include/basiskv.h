@@ -1,0 +1,211 @@
+/*
+ * basiskv.h — C ABI of the BasisKV decode hot path on NVIDIA B200 (sm_100a).
+ *
+ * One decode step of a batch of sequences is four calls on one CUDA stream:
+ *
+ *   basiskv_append       (step 1-2) store each new token's raw key, Value latent
+ *                        and key residual in the paged cache; refresh the
+ *                        summary (mean predicted key) of every page it touched
+ *   basiskv_route        (step 3)   score every page of every sequence for every
+ *                        query head against the summaries; keep the top-k pages
+ *                        plus the sink page and the recent page
+ *   basiskv_decode_attn  (step 4)   exact attention of each query head over the
+ *                        original keys of its selected pages, accumulating the
+ *                        Value latents (rank-r output per head)
+ *   basiskv_out_proj     (step 5)   y = sum_h o_h G_h through the fused factor
+ *
+ * Method: "BasisKV: Value Latents for Communication and Key Routing"
+ * (weekinpapers.com/paper/2611.02583v1, Abstract) and the kongchang.com
+ * explainer of it (sections on binding the Value latent to the output
+ * projection and "用Value潜变量辅助Key路由" on key routing); decode-step order
+ * and attention formula: machinelearning.ru "KV-кэширование", sections
+ * "Фаза Decode" and "Математическая формализация"; paged cache: same page,
+ * section "Форматы хранения и библиотеки".
+ *
+ * Conventions for every entry point
+ *   - Pointers marked (device) are CUDA device pointers owned by the caller;
+ *     the library never allocates, frees or retains them.  Pointers marked
+ *     (host) are read during the call only.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work and return; results are ready when the stream is.
+ *   - Host-side validation failures return an error status and launch
+ *     nothing.  No C++ exception crosses the ABI.
+ *   - Faults the kernels can detect (a block-table entry or selected page out
+ *     of range, a sequence length that cannot hold the new tokens, a wait that
+ *     timed out) are OR-ed into *err_flag (device int32, bit values
+ *     BASISKV_DEVERR_*) and the offending page or sequence is skipped; no
+ *     kernel traps.  The caller zeroes the flag and reads it when it likes.
+ *   - Tensor layouts are dense row-major in the order written.  `dtype` in
+ *     basiskv_config fixes the element type of k_raw, c_lat, r_res, q, the
+ *     new tokens and every factor (fp32 or bf16); summaries, o_lat, y and
+ *     scores are always fp32.
+ *   - Query head h uses KV head g(h) = h / (Hq / Hkv).
+ */
+#ifndef BASISKV_H
+#define BASISKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BASISKV_API __attribute__((visibility("default")))
+#else
+#define BASISKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BASISKV_ABI_VERSION 1
+
+typedef enum {
+  BASISKV_OK = 0,
+  BASISKV_ERR_INVALID_ARG = 1,   /* a NULL pointer, a negative size, an inconsistent shape */
+  BASISKV_ERR_UNSUPPORTED = 2,   /* a valid shape this build has no kernel for            */
+  BASISKV_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed                 */
+  BASISKV_ERR_WORKSPACE = 4      /* workspace NULL or smaller than basiskv_workspace_bytes */
+} basiskv_status;
+
+typedef enum { BASISKV_F32 = 0, BASISKV_BF16 = 1 } basiskv_dtype;
+
+/* Bits OR-ed into *err_flag by the kernels. */
+#define BASISKV_DEVERR_BLOCK_TABLE 1   /* block_table entry outside [0, num_phys_pages)      */
+#define BASISKV_DEVERR_SELECTION 2     /* sel entry outside [0, pages of the sequence)       */
+#define BASISKV_DEVERR_SEQ_LEN 4       /* seq_len < n_new, or > max_pages * page_size         */
+#define BASISKV_DEVERR_TIMEOUT 8       /* an in-kernel wait on a bulk copy gave up (~1 s)     */
+
+/*
+ * Shapes.  Supported by this build: head_dim in {64, 128}; page_size in
+ * {16, 32, 64}; 1 <= rank_v <= 128; 1 <= rank_k <= 64;
+ * Hq / Hkv in {1, 2, 4, 8}; 1 <= top_k and top_k + 2 <= 1024;
+ * hidden a multiple of 16.  Anything else returns BASISKV_ERR_UNSUPPORTED.
+ */
+typedef struct {
+  int32_t num_q_heads;   /* Hq                                          */
+  int32_t num_kv_heads;  /* Hkv (KV heads; Hq % Hkv == 0)                */
+  int32_t head_dim;      /* d                                           */
+  int32_t rank_v;        /* r: Value-latent rank                         */
+  int32_t rank_k;        /* s: key-residual rank                         */
+  int32_t page_size;     /* P: tokens per page                           */
+  int32_t hidden;        /* width of the layer output y                  */
+  int32_t top_k;         /* k: routed pages per head, sink/recent excluded */
+  int32_t dtype;         /* basiskv_dtype                                */
+} basiskv_config;
+
+/*
+ * Paged cache (device).  A physical page holds, for every KV head, one
+ * contiguous block per tensor:
+ *   k_raw   [num_phys_pages][Hkv][P][d]   original keys (dtype)
+ *   c_lat   [num_phys_pages][Hkv][P][r]   Value latents C = v A_g (dtype)
+ *   r_res   [num_phys_pages][Hkv][P][s]   key residuals R = (k - C P_g) E_g (dtype)
+ *   summary [num_phys_pages][Hkv][d]      mean predicted key of the page (fp32)
+ * block_table [B][max_pages] maps logical page p of sequence b to a physical
+ * page; seq_len [B] is each sequence's token count AFTER the step's append.
+ * Sequence b has n_b = ceil(seq_len[b] / P) pages; the recent page n_b - 1
+ * may be partial and only its first seq_len[b] - (n_b - 1) P slots are valid.
+ */
+typedef struct {
+  void* k_raw;
+  void* c_lat;
+  void* r_res;
+  float* summary;
+  const int32_t* block_table;
+  const int32_t* seq_len;
+  int32_t num_phys_pages;
+  int32_t max_pages;
+} basiskv_cache;
+
+/*
+ * Factors (device, dtype).  A [Hkv][d][r] (Value -> latent), P [Hkv][r][d]
+ * (latent -> predicted key), E [Hkv][d][s] (key residual basis),
+ * Gt [hidden][Hq][r]: the fused out-projection factor G_h = B_g(h) W_O,h,
+ * stored transposed (row c holds output column c for every head and latent
+ * dimension); basiskv_fuse_out_factor writes it.
+ */
+typedef struct {
+  const void* A;
+  const void* P;
+  const void* E;
+  const void* Gt;
+} basiskv_factors;
+
+/*
+ * Steps 1-2.  Append n_new tokens to each of `batch` sequences.
+ * k_new, v_new (device, dtype): [batch][n_new][Hkv][d]; token t of sequence b
+ * lands at position seq_len[b] - n_new + t (the pages it needs must already be
+ * in block_table).  Per token and KV head g: C = v A_g, R = (k - C P_g) E_g
+ * (R from the unrounded C), accumulated in fp64 and rounded once to dtype;
+ * the raw key is stored as given.  Then every touched page's summary is
+ * recomputed over its valid tokens: S = mean(C) P_g + mean(R) E_g^T, rounded
+ * to fp32.  n_new = 1 is the decode step; larger n_new is prefill.
+ * err_flag (device int32) may not be NULL.
+ */
+BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* cache,
+                              const basiskv_factors* factors, const void* k_new,
+                              const void* v_new, int32_t batch, int32_t n_new,
+                              int32_t* err_flag, void* stream);
+
+/*
+ * Step 3.  Page routing for every (sequence, query head).
+ * q (device, dtype) [batch][Hq][d].  score_p = q_h . S_p in fp32 over every
+ * logical page.  If n_b <= top_k + 2 every page is selected; otherwise pages
+ * 0 and n_b - 1 plus the top_k of pages 1..n_b-2 under the order (score
+ * descending, page index ascending).
+ * Outputs (device): sel [batch][Hq][top_k + 2] int32 logical page indices in
+ * ascending order, padded with -1; sel_cnt [batch][Hq] int32.
+ * scores (device, optional, may be NULL): [batch][Hq][max_pages] fp32, the
+ * score of every page p < n_b (others untouched).
+ * workspace (device): at least basiskv_workspace_bytes(cfg, batch, max_pages)
+ * bytes; contents need no initialisation and are clobbered.
+ */
+BASISKV_API basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache,
+                             const void* q, int32_t batch, int32_t* sel, int32_t* sel_cnt,
+                             float* scores, void* workspace, size_t workspace_bytes,
+                             int32_t* err_flag, void* stream);
+
+/*
+ * Step 4.  Exact sparse attention.  For each (b, h): over the valid tokens j
+ * of the pages in sel[b][h][0 .. sel_cnt-1], s_j = q_h . K_j / sqrt(d) on the
+ * original keys, w = softmax(s), o_lat[b][h] = sum_j w_j C_j (fp32, [batch][Hq][r]).
+ * Pages selected by several query heads of one KV head are read once.
+ * sel / sel_cnt as written by basiskv_route (any ascending, duplicate-free
+ * list of valid pages is accepted).  workspace as for basiskv_route (the same
+ * buffer may be passed to both).  err_flag may not be NULL.
+ */
+BASISKV_API basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,
+                                   const void* q, int32_t batch, const int32_t* sel,
+                                   const int32_t* sel_cnt, float* o_lat, void* workspace,
+                                   size_t workspace_bytes, int32_t* err_flag, void* stream);
+
+/*
+ * Step 5.  y[b] = sum_h o_lat[b][h] G_h (fp32 [batch][hidden]) with G read from
+ * factors->Gt.  The full Value width is never formed.  workspace as above.
+ */
+BASISKV_API basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors* factors,
+                                const float* o_lat, int32_t batch, float* y, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
+ * Weight preparation for step 5 (not per step).  Gt[c][h][i] =
+ * sum_j Bf[g(h)][i][j] W_O[h d + j][c], accumulated in fp64 and rounded once to
+ * dtype.  Bf (device, dtype) [Hkv][r][d]; W_O (device, dtype) [Hq d][hidden];
+ * Gt (device, dtype) [hidden][Hq][r].
+ */
+BASISKV_API basiskv_status basiskv_fuse_out_factor(const basiskv_config* cfg, const void* Bf,
+                                       const void* W_O, void* Gt, void* stream);
+
+/* Workspace bytes needed by route / decode_attn / out_proj for this shape. */
+BASISKV_API size_t basiskv_workspace_bytes(const basiskv_config* cfg, int32_t batch, int32_t max_pages);
+
+/* Static description of a status code (never NULL). */
+BASISKV_API const char* basiskv_status_string(int32_t status);
+
+/* BASISKV_ABI_VERSION of the loaded library. */
+BASISKV_API int32_t basiskv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASISKV_H */

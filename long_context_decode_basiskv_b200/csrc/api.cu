@@ -1,0 +1,202 @@
+// C ABI entry points (include/basiskv.h): host-side validation, workspace
+// layout and kernel dispatch.  Nothing here allocates device memory.
+#include <stdio.h>
+
+#include "kernels.cuh"
+
+namespace bkv {
+
+// ---------------------------------------------------------------------------
+// helpers
+// ---------------------------------------------------------------------------
+constexpr int kMaxPagesLimit = 49152;  // route select keeps one key per page in shared memory
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int esize(const basiskv_config* c) { return c->dtype == BASISKV_BF16 ? 2 : 4; }
+
+static basiskv_status check_config(const basiskv_config* c) {
+  if (!c) return BASISKV_ERR_INVALID_ARG;
+  if (c->num_q_heads <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0 || c->rank_v <= 0 ||
+      c->rank_k <= 0 || c->page_size <= 0 || c->hidden <= 0 || c->top_k <= 0)
+    return BASISKV_ERR_INVALID_ARG;
+  if (c->num_q_heads % c->num_kv_heads != 0) return BASISKV_ERR_INVALID_ARG;
+  if (c->dtype != BASISKV_F32 && c->dtype != BASISKV_BF16) return BASISKV_ERR_INVALID_ARG;
+  if (c->rank_v > c->head_dim || c->rank_k > c->head_dim) return BASISKV_ERR_INVALID_ARG;
+  const int G = c->num_q_heads / c->num_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return BASISKV_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return BASISKV_ERR_UNSUPPORTED;
+  if (c->page_size != 16 && c->page_size != 32 && c->page_size != 64) return BASISKV_ERR_UNSUPPORTED;
+  if (c->rank_v > 128 || c->rank_k > 64) return BASISKV_ERR_UNSUPPORTED;
+  if (c->top_k + 2 > 1024) return BASISKV_ERR_UNSUPPORTED;
+  if (c->hidden % 16 != 0) return BASISKV_ERR_UNSUPPORTED;
+  if (((size_t)c->num_q_heads * c->rank_v * esize(c)) % 16 != 0) return BASISKV_ERR_UNSUPPORTED;
+  return BASISKV_OK;
+}
+
+static basiskv_status check_cache(const basiskv_config* c, const basiskv_cache* k, bool need_res) {
+  if (!k || !k->k_raw || !k->c_lat || !k->summary || !k->block_table || !k->seq_len)
+    return BASISKV_ERR_INVALID_ARG;
+  if (need_res && !k->r_res) return BASISKV_ERR_INVALID_ARG;
+  if (k->num_phys_pages <= 0 || k->max_pages <= 0) return BASISKV_ERR_INVALID_ARG;
+  if (k->max_pages > kMaxPagesLimit) return BASISKV_ERR_UNSUPPORTED;
+  if (!aligned16(k->k_raw) || !aligned16(k->c_lat) || !aligned16(k->summary) ||
+      (need_res && !aligned16(k->r_res)))
+    return BASISKV_ERR_INVALID_ARG;
+  (void)c;
+  return BASISKV_OK;
+}
+
+static int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+struct Workspace {
+  size_t scores, uni, ucnt, part, total;
+  int umax, nsplit, pps;
+};
+
+static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static Workspace layout(const basiskv_config* c, int batch, int max_pages) {
+  Workspace w{};
+  const int G = c->num_q_heads / c->num_kv_heads;
+  long long um = (long long)G * (c->top_k + 2);
+  if (um > max_pages) um = max_pages;
+  w.umax = (int)um;
+  w.pps = attn_pages_per_split(c->page_size);
+  w.nsplit = attn_nsplit(w.umax, c->page_size);
+  size_t off = 0;
+  w.scores = off;
+  off += up256((size_t)batch * c->num_q_heads * max_pages * 4);
+  w.uni = off;
+  off += up256((size_t)batch * c->num_kv_heads * w.umax * 4);
+  w.ucnt = off;
+  off += up256((size_t)batch * c->num_kv_heads * 4);
+  w.part = off;
+  off += up256((size_t)batch * c->num_q_heads * w.nsplit * (c->rank_v + 2) * 4);
+  w.total = off;
+  return w;
+}
+
+static basiskv_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return BASISKV_OK;
+  fprintf(stderr, "basiskv: CUDA error %s\n", cudaGetErrorString(e));
+  return BASISKV_ERR_CUDA;
+}
+
+}  // namespace bkv
+
+using namespace bkv;
+
+extern "C" {
+
+int32_t basiskv_abi_version(void) { return BASISKV_ABI_VERSION; }
+
+const char* basiskv_status_string(int32_t s) {
+  switch (s) {
+    case BASISKV_OK: return "ok";
+    case BASISKV_ERR_INVALID_ARG: return "invalid argument";
+    case BASISKV_ERR_UNSUPPORTED: return "unsupported shape";
+    case BASISKV_ERR_CUDA: return "CUDA error";
+    case BASISKV_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+size_t basiskv_workspace_bytes(const basiskv_config* cfg, int32_t batch, int32_t max_pages) {
+  if (check_config(cfg) != BASISKV_OK || batch < 0 || max_pages <= 0) return 0;
+  return layout(cfg, batch, max_pages).total;
+}
+
+basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* cache,
+                              const basiskv_factors* f, const void* k_new, const void* v_new,
+                              int32_t batch, int32_t n_new, int32_t* err_flag, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != BASISKV_OK) return s;
+  if (batch == 0 || n_new == 0) return BASISKV_OK;
+  if (!f || !f->A || !f->P || !f->E || !k_new || !v_new || !err_flag || batch < 0 || n_new < 0)
+    return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(f->A) || !aligned16(f->P) || !aligned16(f->E)) return BASISKV_ERR_INVALID_ARG;
+  if ((long long)n_new > (long long)cache->max_pages * cfg->page_size) return BASISKV_ERR_INVALID_ARG;
+  AppendParams p{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
+                 cache->summary, cache->block_table, cache->seq_len, err_flag,
+                 batch, n_new, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
+                 cfg->page_size, cache->max_pages, cache->num_phys_pages};
+  return cuda_status(launch_append(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
+}
+
+basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
+                             int32_t batch, int32_t* sel, int32_t* sel_cnt, float* scores,
+                             void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if ((s = check_cache(cfg, cache, false)) != BASISKV_OK) return s;
+  if (batch == 0) return BASISKV_OK;
+  if (!q || !sel || !sel_cnt || !err_flag || batch < 0) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || (scores && !aligned16(scores))) return BASISKV_ERR_INVALID_ARG;
+  const Workspace w = layout(cfg, batch, cache->max_pages);
+  if (!ws || ws_bytes < w.total || !aligned16(ws)) return BASISKV_ERR_WORKSPACE;
+  float* sc = scores ? scores : reinterpret_cast<float*>(static_cast<char*>(ws) + w.scores);
+  ScoreParams sp{q, cache->summary, cache->block_table, cache->seq_len, sc, err_flag,
+                 batch, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cache->max_pages,
+                 cache->num_phys_pages, (cache->max_pages + 7) / 8};
+  SelectParams selp{sc, cache->seq_len, sel, sel_cnt, cfg->num_q_heads, cfg->page_size,
+                    cache->max_pages, cfg->top_k};
+  return cuda_status(launch_route(sp, selp, cfg->head_dim, cfg->num_q_heads / cfg->num_kv_heads,
+                                  cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream));
+}
+
+basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,
+                                   const void* q, int32_t batch, const int32_t* sel,
+                                   const int32_t* sel_cnt, float* o_lat, void* ws, size_t ws_bytes,
+                                   int32_t* err_flag, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if ((s = check_cache(cfg, cache, false)) != BASISKV_OK) return s;
+  if (batch == 0) return BASISKV_OK;
+  if (!q || !sel || !sel_cnt || !o_lat || !err_flag || batch < 0) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(q)) return BASISKV_ERR_INVALID_ARG;
+  const Workspace w = layout(cfg, batch, cache->max_pages);
+  if (!ws || ws_bytes < w.total || !aligned16(ws)) return BASISKV_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  int32_t* uni = reinterpret_cast<int32_t*>(base + w.uni);
+  int32_t* ucnt = reinterpret_cast<int32_t*>(base + w.ucnt);
+  float* part = reinterpret_cast<float*>(base + w.part);
+  UnionParams up{sel, sel_cnt, cache->seq_len, uni, ucnt, err_flag, cfg->num_q_heads,
+                 cfg->num_kv_heads, cfg->page_size, cache->max_pages, cfg->top_k, w.umax};
+  AttnParams ap{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, uni, ucnt, part,
+                err_flag, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v,
+                cache->max_pages, cache->num_phys_pages, w.umax, w.pps, w.nsplit,
+                (float)(1.4426950408889634 / sqrt((double)cfg->head_dim)), 0};
+  CombineParams cp{part, ucnt, o_lat, cfg->num_q_heads, cfg->num_kv_heads, cfg->rank_v, w.pps, w.nsplit};
+  return cuda_status(launch_decode_attn(up, ap, cp, batch, cfg->head_dim, cfg->dtype == BASISKV_BF16,
+                                        (cudaStream_t)stream));
+}
+
+basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors* f, const float* o_lat,
+                                int32_t batch, float* y, void* ws, size_t ws_bytes, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if (batch == 0) return BASISKV_OK;
+  if (!f || !f->Gt || !o_lat || !y || batch < 0) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(f->Gt) || !aligned16(o_lat) || !aligned16(y)) return BASISKV_ERR_INVALID_ARG;
+  (void)ws;
+  (void)ws_bytes;
+  OutProjParams p{o_lat, f->Gt, y, batch, cfg->num_q_heads * cfg->rank_v, cfg->hidden};
+  return cuda_status(launch_out_proj_gemv(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
+}
+
+basiskv_status basiskv_fuse_out_factor(const basiskv_config* cfg, const void* Bf, const void* W_O,
+                                       void* Gt, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if (!Bf || !W_O || !Gt) return BASISKV_ERR_INVALID_ARG;
+  FuseParams p{Bf, W_O, Gt, cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->hidden};
+  return cuda_status(launch_fuse(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
+}
+
+}  // extern "C"

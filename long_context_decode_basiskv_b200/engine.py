@@ -1,0 +1,94 @@
+"""One decode step of BasisKV on the GPU, driven through the C ABI.
+
+``DecodeEngine`` owns the device state of a batch: the paged cache (built by
+the library's own append kernel in prefill mode), the factors with the fused
+out-projection factor (built by the library's fusion kernel), the step's
+inputs and outputs, and one workspace.  ``step()`` enqueues the four calls of
+one decode step: append, route, decode_attn, out_proj.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as bk
+from .workloads import Case
+
+
+def config_of(case: Case) -> bk.Config:
+    wl = case.wl
+    return bk.Config(wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.rank_v, wl.rank_k,
+                     wl.page_size, wl.hidden, wl.top_k, wl.torch_dtype)
+
+
+class DecodeEngine:
+    def __init__(self, case: Case, device="cuda", stream=None):
+        self.case = case
+        self.cfg = cfg = config_of(case)
+        self.device = torch.device(device)
+        dev = self.device
+        B = case.wl.batch
+        lengths = torch.tensor(case.lengths, dtype=torch.int32)
+        self.cache = bk.PagedCache(cfg, case.num_phys_pages, case.block_table, lengths, device=dev)
+        self.factors = bk.Factors(case.A.to(dev).contiguous(), case.P.to(dev).contiguous(),
+                                  case.E.to(dev).contiguous(),
+                                  torch.empty((cfg.hidden, cfg.num_q_heads, cfg.rank_v),
+                                              dtype=cfg.dtype, device=dev))
+        bk.fuse_out_factor(cfg, case.Bf.to(dev).contiguous(), case.W_O.to(dev).contiguous(),
+                           self.factors.Gt, stream)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.ws = bk.alloc_workspace(cfg, B, self.cache.max_pages, device=dev)
+        # step inputs: the last token of every sequence, and the query
+        self.k_new = torch.stack([k[-1] for k in case.keys]).unsqueeze(1).to(dev).contiguous()
+        self.v_new = torch.stack([v[-1] for v in case.values]).unsqueeze(1).to(dev).contiguous()
+        self.q = case.q.to(dev).contiguous()
+        # step outputs
+        self.sel = torch.empty((B, cfg.num_q_heads, cfg.top_k + 2), dtype=torch.int32, device=dev)
+        self.sel_cnt = torch.empty((B, cfg.num_q_heads), dtype=torch.int32, device=dev)
+        self.o_lat = torch.empty((B, cfg.num_q_heads, cfg.rank_v), dtype=torch.float32, device=dev)
+        self.y = torch.empty((B, cfg.hidden), dtype=torch.float32, device=dev)
+        self.prefill(stream)
+
+    def prefill(self, stream=None):
+        """Append every token but the last of each sequence (one call per sequence)."""
+        cfg, case = self.cfg, self.case
+        dev = self.device
+        for b, L in enumerate(case.lengths):
+            if L <= 1:
+                continue
+            sub = bk.PagedCache.__new__(bk.PagedCache)
+            sub.__dict__.update(self.cache.__dict__)
+            sub.block_table = self.cache.block_table[b:b + 1]
+            sub.seq_len = torch.tensor([L - 1], dtype=torch.int32, device=dev)
+            k = case.keys[b][:-1].to(dev).unsqueeze(0).contiguous()
+            v = case.values[b][:-1].to(dev).unsqueeze(0).contiguous()
+            bk.append(cfg, sub, self.factors, k, v, self.err, stream)
+
+    def append(self, stream=None):
+        bk.append(self.cfg, self.cache, self.factors, self.k_new, self.v_new, self.err, stream)
+
+    def route(self, scores=None, stream=None):
+        bk.route(self.cfg, self.cache, self.q, self.sel, self.sel_cnt, self.ws, self.err, scores, stream)
+
+    def decode_attn(self, stream=None):
+        bk.decode_attn(self.cfg, self.cache, self.q, self.sel, self.sel_cnt, self.o_lat, self.ws,
+                       self.err, stream)
+
+    def out_proj(self, stream=None):
+        bk.out_proj(self.cfg, self.factors, self.o_lat, self.y, self.ws, stream)
+
+    def step(self, stream=None):
+        """One decode step: append -> route -> decode_attn -> out_proj (one stream)."""
+        self.append(stream)
+        self.route(stream=stream)
+        self.decode_attn(stream)
+        self.out_proj(stream)
+        return self.y
+
+    def logical(self, tensor: torch.Tensor, b: int) -> torch.Tensor:
+        """Gather a per-page cache tensor [phys, Hkv, P, x] of sequence b into [Hkv, L, x]."""
+        L = self.case.lengths[b]
+        n = -(-L // self.cfg.page_size)
+        phys = self.cache.block_table[b, :n].long()
+        t = tensor[phys]                       # [n, Hkv, P, x]
+        t = t.permute(1, 0, 2, 3).reshape(t.shape[1], n * self.cfg.page_size, -1)
+        return t[:, :L]

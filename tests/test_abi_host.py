@@ -1,0 +1,104 @@
+"""The C ABI library on the host (no GPU needed): it loads, exports every
+function include/basiskv.h declares, and its host-side validation rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decode_basiskv_b200 import binding as bk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "basiskv.h")).read()
+    return sorted(set(re.findall(r"BASISKV_API\s+[\w\s\*]+?\b(basiskv_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(bk.LIB_PATH):
+        from long_context_decode_basiskv_b200 import build
+        build.build()
+    return bk.lib()
+
+
+def test_header_declarations_match_binding():
+    assert _declared() == sorted(bk.SYMBOLS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings(L):
+    assert L.basiskv_abi_version() == 1
+    assert L.basiskv_status_string(0) == b"ok"
+    assert L.basiskv_status_string(4).startswith(b"workspace")
+    assert L.basiskv_status_string(99) == b"unknown status"
+
+
+def _cfg(**kw):
+    base = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, rank_v=64, rank_k=32, page_size=16,
+                hidden=4096, top_k=128, dtype=bk.BF16)
+    base.update(kw)
+    return bk.CConfig(*[base[f] for f, _ in bk.CConfig._fields_])
+
+
+def test_workspace_bytes(L):
+    n = L.basiskv_workspace_bytes(ctypes.byref(_cfg()), 8, 2048)
+    assert n >= 8 * 32 * 2048 * 4          # at least the routing scores
+    assert L.basiskv_workspace_bytes(ctypes.byref(_cfg(head_dim=96)), 8, 2048) == 0
+    assert L.basiskv_workspace_bytes(None, 8, 2048) == 0
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(num_q_heads=30), bk.ERR_INVALID_ARG),        # Hq % Hkv != 0
+    (dict(head_dim=96), bk.ERR_UNSUPPORTED),
+    (dict(page_size=8), bk.ERR_UNSUPPORTED),
+    (dict(rank_v=0), bk.ERR_INVALID_ARG),
+    (dict(top_k=1023), bk.ERR_UNSUPPORTED),
+    (dict(num_q_heads=48, num_kv_heads=3), bk.ERR_UNSUPPORTED),   # G = 16
+    (dict(dtype=7), bk.ERR_INVALID_ARG),
+])
+def test_config_validation(L, bad, status):
+    cfg = _cfg(**bad)
+    cache = bk.CCache(16, 16, 16, 16, 16, 16, 10, 10)   # never dereferenced: validation fails first
+    st = L.basiskv_route(ctypes.byref(cfg), ctypes.byref(cache), 16, 1, 16, 16, None, 16, 1 << 30, 16, None)
+    assert st == status
+
+
+def test_null_and_misaligned_pointers(L):
+    cfg = _cfg()
+    good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    assert L.basiskv_route(ctypes.byref(cfg), None, 256, 1, 256, 256, None, 256, 1 << 30, 256, None) == bk.ERR_INVALID_ARG
+    misaligned = bk.CCache(264, 256, 256, 256, 256, 256, 10, 10)
+    assert L.basiskv_route(ctypes.byref(cfg), ctypes.byref(misaligned), 256, 1, 256, 256, None, 256,
+                           1 << 30, 256, None) == bk.ERR_INVALID_ARG
+    # workspace too small
+    assert L.basiskv_route(ctypes.byref(cfg), ctypes.byref(good), 256, 1, 256, 256, None, 256, 16, 256,
+                           None) == bk.ERR_WORKSPACE
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(good), 256, 1, 256, 256, 256, None, 0,
+                                 256, None) == bk.ERR_WORKSPACE
+    # err flag required
+    f = bk.CFactors(256, 256, 256, 256)
+    assert L.basiskv_append(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 1, 1, None,
+                            None) == bk.ERR_INVALID_ARG
+    # too many pages for the routing kernel
+    big = bk.CCache(256, 256, 256, 256, 256, 256, 10, 1 << 20)
+    assert L.basiskv_route(ctypes.byref(cfg), ctypes.byref(big), 256, 1, 256, 256, None, 256, 1 << 40, 256,
+                           None) == bk.ERR_UNSUPPORTED
+
+
+def test_empty_batch_is_a_no_op(L):
+    cfg = _cfg()
+    good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    f = bk.CFactors(256, 256, 256, 256)
+    assert L.basiskv_append(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 0, 1, 256,
+                            None) == bk.OK
+    assert L.basiskv_route(ctypes.byref(cfg), ctypes.byref(good), 256, 0, 256, 256, None, None, 0, 256,
+                           None) == bk.OK
+    assert L.basiskv_out_proj(ctypes.byref(cfg), ctypes.byref(f), 256, 0, 256, None, 0, None) == bk.OK
