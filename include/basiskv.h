@@ -179,6 +179,31 @@ BASISKV_API basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const 
                                    size_t workspace_bytes, int32_t* err_flag, void* stream);
 
 /*
+ * basiskv_decode_attn without a workspace.  This entry point has no
+ * counterpart in the paper: it exists for callers that cannot allocate
+ * device memory (a plugin whose host engine owns every allocation, code that
+ * runs while its stream is captured into a CUDA graph, a fixed memory budget
+ * after start-up).  It computes exactly what basiskv_decode_attn computes, with
+ * the same arguments minus the workspace, using a scratch array of 16 MiB that
+ * the library keeps in device memory on every GPU where it is loaded, for the
+ * life of the process.
+ *   - Shapes whose scratch (union lists, counts, split partials) exceeds
+ *     16 MiB return BASISKV_ERR_WORKSPACE (with a message on stderr) and
+ *     launch nothing; use basiskv_decode_attn then.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call on a device shares the one array.  Calls that may overlap on
+ *     the GPU (different streams without ordering) race and corrupt each
+ *     other's results; order them.  The scratch needs no initialisation: each
+ *     call writes every part of it that it reads.
+ */
+BASISKV_API basiskv_status basiskv_decode_attn_noalloc(const basiskv_config* cfg,
+                                                       const basiskv_cache* cache, const void* q,
+                                                       int32_t batch, const int32_t* sel,
+                                                       const int32_t* sel_cnt, float* o_lat,
+                                                       int32_t* err_flag, void* stream);
+
+/*
  * Step 5.  y[b] = sum_h o_lat[b][h] G_h (fp32 [batch][hidden]) with G read from
  * factors->Gt.  The full Value width is never formed.  workspace as above.
  */

@@ -25,7 +25,7 @@ DEVERR_BLOCK_TABLE, DEVERR_SELECTION, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 
 SYMBOLS = [
     "basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
     "basiskv_fuse_out_factor", "basiskv_workspace_bytes", "basiskv_status_string",
-    "basiskv_abi_version",
+    "basiskv_abi_version", "basiskv_decode_attn_noalloc",
 ]
 
 
@@ -65,6 +65,7 @@ def lib():
     L.basiskv_route.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, sz, vp, vp]
     L.basiskv_decode_attn.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, sz, vp, vp]
     L.basiskv_out_proj.argtypes = [pc, pf, vp, i32, vp, vp, sz, vp]
+    L.basiskv_decode_attn_noalloc.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, vp]
     L.basiskv_fuse_out_factor.argtypes = [pc, vp, vp, vp, vp]
     L.basiskv_workspace_bytes.argtypes = [pc, i32, i32]
     L.basiskv_workspace_bytes.restype = sz
@@ -72,7 +73,7 @@ def lib():
     L.basiskv_status_string.restype = ctypes.c_char_p
     L.basiskv_abi_version.argtypes = []
     for name in ["basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
-                 "basiskv_fuse_out_factor", "basiskv_abi_version"]:
+                 "basiskv_fuse_out_factor", "basiskv_abi_version", "basiskv_decode_attn_noalloc"]:
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -240,3 +241,18 @@ def out_proj(cfg: Config, f: Factors, o_lat: torch.Tensor, y: torch.Tensor, ws: 
     _need(ws, "workspace", torch.uint8)
     _check(lib().basiskv_out_proj(ctypes.byref(cfg.c()), ctypes.byref(f.c()), _ptr(o_lat), B, _ptr(y),
                                   _ptr(ws), ws.numel(), _stream(stream)), "basiskv_out_proj")
+
+
+def decode_attn_noalloc(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor,
+                        sel_cnt: torch.Tensor, o_lat: torch.Tensor, err: torch.Tensor, stream=None):
+    """decode_attn for callers that cannot allocate: the library's fixed 16 MiB scratch
+    stands in for the workspace (see basiskv_decode_attn_noalloc in include/basiskv.h)."""
+    B = q.shape[0]
+    _need(q, "q", cfg.dtype, (B, cfg.num_q_heads, cfg.head_dim))
+    _need(sel, "sel", torch.int32, (B, cfg.num_q_heads, cfg.top_k + 2))
+    _need(sel_cnt, "sel_cnt", torch.int32, (B, cfg.num_q_heads))
+    _need(o_lat, "o_lat", torch.float32, (B, cfg.num_q_heads, cfg.rank_v))
+    _need(err, "err", torch.int32)
+    _check(lib().basiskv_decode_attn_noalloc(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), _ptr(q), B,
+                                             _ptr(sel), _ptr(sel_cnt), _ptr(o_lat), _ptr(err),
+                                             _stream(stream)), "basiskv_decode_attn_noalloc")

@@ -1,0 +1,123 @@
+// basiskv_decode_attn_noalloc: the sparse-attention call for callers that
+// cannot allocate device memory.
+//
+// Some callers have no way to hand this library a workspace: a plugin whose
+// enqueue hook runs inside a host engine that owns every device allocation,
+// code that runs while a stream is being captured into a CUDA graph (where
+// cudaMalloc is not allowed), or a deployment with a fixed memory budget
+// that forbids allocation after start-up.  This entry point runs exactly the
+// kernels of basiskv_decode_attn, but its scratch (the union lists, their
+// counts and the per-split partial results) lives in one file-scope
+// __device__ array of fixed size that the library owns.  The caller still
+// passes the inputs and the output.
+//
+// The array costs kNoAllocScratchBytes of memory on every GPU on which the
+// library is loaded, until the process exits.
+#include <stdio.h>
+
+#include "kernels.cuh"
+
+namespace bkv {
+
+// Fixed scratch for basiskv_decode_attn_noalloc (16 MiB).
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_addr_mu;
+void* g_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands for the symbol; the address the kernels need
+// is looked up once per device, with that device current.
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_addr_mu);
+  if (!g_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_addr[dev] = p;
+  }
+  *out = g_addr[dev];
+  return cudaSuccess;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+}  // namespace bkv
+
+using namespace bkv;
+
+extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
+    const basiskv_config* cfg, const basiskv_cache* cache, const void* q, int32_t batch,
+    const int32_t* sel, const int32_t* sel_cnt, float* o_lat, int32_t* err_flag, void* stream) {
+  if (!cfg || !cache) return BASISKV_ERR_INVALID_ARG;
+  if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->num_q_heads % cfg->num_kv_heads != 0 ||
+      cfg->rank_v <= 0 || cfg->page_size <= 0 || cfg->top_k <= 0 || batch < 0)
+    return BASISKV_ERR_INVALID_ARG;
+  if (batch == 0) return BASISKV_OK;
+  if (cache->max_pages <= 0) return BASISKV_ERR_INVALID_ARG;
+
+  // the same scratch regions basiskv_decode_attn takes from its workspace
+  const int G = cfg->num_q_heads / cfg->num_kv_heads;
+  long long um = (long long)G * (cfg->top_k + 2);
+  if (um > cache->max_pages) um = cache->max_pages;
+  const int umax = (int)um;
+  const int pps = attn_pages_per_split(cfg->page_size);
+  const int nsplit = attn_nsplit(umax, cfg->page_size);
+  const size_t uni_off = 0;
+  const size_t ucnt_off = uni_off + up256((size_t)batch * cfg->num_kv_heads * umax * 4);
+  const size_t part_off = ucnt_off + up256((size_t)batch * cfg->num_kv_heads * 4);
+  const size_t need = part_off + up256((size_t)batch * cfg->num_q_heads * nsplit * (cfg->rank_v + 2) * 4);
+  if (need > kNoAllocScratchBytes) {
+    fprintf(stderr,
+            "basiskv_decode_attn_noalloc: this shape needs %zu bytes of scratch, more than the "
+            "fixed %zu; use basiskv_decode_attn with a workspace\n",
+            need, kNoAllocScratchBytes);
+    return BASISKV_ERR_WORKSPACE;
+  }
+
+  // the remaining checks of basiskv_decode_attn: a supported shape (the
+  // workspace query returns 0 otherwise), pointers present and aligned
+  if (basiskv_workspace_bytes(cfg, batch, cache->max_pages) == 0) return BASISKV_ERR_UNSUPPORTED;
+  if (!q || !sel || !sel_cnt || !o_lat || !err_flag) return BASISKV_ERR_INVALID_ARG;
+  if (!cache->k_raw || !cache->c_lat || !cache->block_table || !cache->seq_len ||
+      cache->num_phys_pages <= 0)
+    return BASISKV_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(cache->k_raw) |
+       reinterpret_cast<uintptr_t>(cache->c_lat)) & 15u)
+    return BASISKV_ERR_INVALID_ARG;
+
+  void* scratch = nullptr;
+  cudaError_t e = scratch_address(&scratch);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "basiskv_decode_attn_noalloc: cudaGetSymbolAddress failed: %s\n",
+            cudaGetErrorString(e));
+    return BASISKV_ERR_CUDA;
+  }
+  char* base = static_cast<char*>(scratch);
+  int32_t* uni = reinterpret_cast<int32_t*>(base + uni_off);
+  int32_t* ucnt = reinterpret_cast<int32_t*>(base + ucnt_off);
+  float* part = reinterpret_cast<float*>(base + part_off);
+  UnionParams up{sel, sel_cnt, cache->seq_len, uni, ucnt, err_flag, cfg->num_q_heads,
+                 cfg->num_kv_heads, cfg->page_size, cache->max_pages, cfg->top_k, umax};
+  AttnParams ap{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, uni, ucnt, part,
+                err_flag, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v,
+                cache->max_pages, cache->num_phys_pages, umax, pps, nsplit,
+                (float)(1.4426950408889634 / sqrt((double)cfg->head_dim)), 0};
+  CombineParams cp{part, ucnt, o_lat, cfg->num_q_heads, cfg->num_kv_heads, cfg->rank_v, pps, nsplit};
+  e = launch_decode_attn(up, ap, cp, batch, cfg->head_dim, cfg->dtype == BASISKV_BF16,
+                         (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "basiskv_decode_attn_noalloc: CUDA error %s\n", cudaGetErrorString(e));
+    return BASISKV_ERR_CUDA;
+  }
+  return BASISKV_OK;
+}
