@@ -186,7 +186,11 @@ basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors
   if (!aligned16(f->Gt) || !aligned16(o_lat) || !aligned16(y)) return BASISKV_ERR_INVALID_ARG;
   (void)ws;
   (void)ws_bytes;
-  OutProjParams p{o_lat, f->Gt, y, batch, cfg->num_q_heads * cfg->rank_v, cfg->hidden};
+  const int K = cfg->num_q_heads * cfg->rank_v;
+  if (cfg->dtype == BASISKV_BF16 && out_proj_tc_supported(K, cfg->hidden, batch))
+    return cuda_status(launch_out_proj_tc(o_lat, f->Gt, y, nullptr, batch, K, cfg->hidden, num_sms(),
+                                          (cudaStream_t)stream));
+  OutProjParams p{o_lat, f->Gt, y, batch, K, cfg->hidden};
   return cuda_status(launch_out_proj_gemv(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
 }
 

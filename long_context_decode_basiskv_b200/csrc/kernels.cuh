@@ -83,6 +83,9 @@ struct OutProjParams {
   int batch, K, hidden;
 };
 cudaError_t launch_out_proj_gemv(const OutProjParams& p, bool bf16, cudaStream_t st);
+bool out_proj_tc_supported(int K, int hidden, int batch);
+cudaError_t launch_out_proj_tc(const float* o, const void* Gt, float* y, int32_t* err, int batch, int K, int hidden,
+                               int num_sms, cudaStream_t st);
 
 struct FuseParams {
   const void* Bf;

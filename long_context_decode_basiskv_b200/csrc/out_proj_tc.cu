@@ -1,0 +1,389 @@
+// Step 5 on the tensor cores: y^T = Gt . o^T with tcgen05 (sm_100a).
+//
+// The fused factor Gt [hidden][K] (K = Hq*r, K-major rows) is the A operand
+// (M = 128 output columns per CTA), the rank-r attention outputs o [B][K] are
+// the B operand (N = batch rows, padded to a multiple of 16).  o is fp32; it
+// is split on the fly into bf16 hi + lo (o ~ hi + lo to ~2^-16 relative) and
+// both halves are multiplied into the same fp32 TMEM accumulator, so the
+// product keeps fp32-level accuracy with bf16 operands.
+//
+// Per CTA: warp 0 streams 128x64 tiles of Gt with 2-D TMA (128-byte swizzle,
+// no multicast) into a 4-stage ring and one of its threads issues the
+// tcgen05.mma instructions; warps 1-4 write the swizzled bf16 hi/lo tiles of
+// o into a matching ring and, at the end, read the accumulator out of TMEM.
+// The K dimension is split over the CTAs of a thread-block cluster; their
+// partial tiles are summed through distributed shared memory in a fixed
+// order (deterministic), each CTA writing a slice of the output rows.
+// HBM-bound: Gt is read once (16.8 MB for the 32K Llama-3-8B shape).
+#include <cuda.h>
+#include <stdio.h>
+
+#include <tuple>
+
+#include "kernels.cuh"
+
+namespace bkv {
+
+constexpr int kTcM = 128;        // output columns (rows of Gt) per CTA
+constexpr int kTcK = 64;         // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 160;  // warp 0: TMA + MMA; warps 1-4: o producers + epilogue
+constexpr uint32_t kTcABytes = kTcM * kTcK * 2;
+
+struct OutProjTcParams {
+  const float* o;  // [B][K]
+  float* y;        // [B][hidden]
+  int32_t* err;
+  int batch, K, hidden, chunks_per_cta, ksplit;
+};
+
+// ---- PTX wrappers ------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// K-major operand tile in shared memory, 128-byte swizzle: rows of 128 bytes,
+// 8-row groups 1024 bytes apart.  Start address advanced by 32 bytes per
+// K = 16 slice inside the swizzle atom.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* base) {
+  const uint64_t addr = smem_u32(base);
+  return ((addr >> 4) & 0x3fffull) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// kind::f16 instruction descriptor: bf16 A and B, fp32 D, both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    out_proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, OutProjTcParams p) {
+  constexpr int S = kTcStages;
+  constexpr uint32_t kBBytes = NB * kTcK * 2;  // one of hi / lo per stage
+  constexpr uint32_t kCols = NB <= 32 ? 32 : 64;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = smem;
+  unsigned char* sB = smem + S * kTcABytes;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(sB + S * 2 * kBBytes);
+  uint64_t* bfull = afull + S;
+  uint64_t* empty = bfull + S;
+  uint64_t* done = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  float* red = reinterpret_cast<float*>(smem);  // [128][NB], reuses the A ring after the last MMA
+  __shared__ int s_fail;  // a bounded wait gave up: the outputs of this cluster become NaN
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int c0 = blockIdx.y * kTcM;
+  const int b0 = blockIdx.z * NB;
+  const int KC = p.K / kTcK;
+  const int ch0 = (int)rank * p.chunks_per_cta;
+  const int nst = max(0, min(KC, ch0 + p.chunks_per_cta) - ch0);
+
+  if (threadIdx.x == 0) s_fail = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) {
+        mbar_init(&afull[s], 1);
+        mbar_init(&bfull[s], 128);
+        mbar_init(&empty[s], 1);
+      }
+      mbar_init(done, 1);
+      fence_mbar_init();
+    }
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0 && nst > 0) {
+      constexpr uint32_t idesc = idesc_bf16(kTcM, NB);
+      for (int i = 0; i < min(S, nst); ++i) {
+        mbar_arrive_expect_tx(&afull[i], kTcABytes);
+        tma_load_2d(sA + i * kTcABytes, &tmA, (ch0 + i) * kTcK, c0, &afull[i]);
+      }
+      for (int i = 0; i < nst && ok; ++i) {
+        const int s = i % S;
+        const uint32_t ph = (uint32_t)((i / S) & 1);
+        if (!mbar_wait_bounded(&afull[s], ph) || !mbar_wait_bounded(&bfull[s], ph)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint64_t ad = smem_desc_sw128(sA + s * kTcABytes);
+        const uint64_t bh = smem_desc_sw128(sB + s * 2 * kBBytes);
+        const uint64_t bl = smem_desc_sw128(sB + s * 2 * kBBytes + kBBytes);
+#pragma unroll
+        for (int j = 0; j < kTcK / 16; ++j) {
+          const uint64_t step = (uint64_t)(j * 32) >> 4;  // 32 bytes per K = 16 slice
+          tc_mma(tmem, ad + step, bh + step, idesc, (i > 0 || j > 0) ? 1u : 0u);
+          tc_mma(tmem, ad + step, bl + step, idesc, 1u);
+        }
+        tc_commit(&empty[s]);
+        if (i + S < nst) {
+          if (!mbar_wait_bounded(&empty[s], ph)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&afull[s], kTcABytes);
+          tma_load_2d(sA + s * kTcABytes, &tmA, (ch0 + i + S) * kTcK, c0, &afull[s]);
+        }
+      }
+      tc_commit(done);  // arrives when every MMA issued above has completed
+    }
+    __syncwarp();
+  } else {
+    // o producers: 128 threads write the bf16 hi / lo tiles of stage i
+    const int t = threadIdx.x - 32;
+    for (int i = 0; i < nst && ok; ++i) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / S) - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      const int kc = ch0 + i;
+      unsigned char* hi_t = sB + s * 2 * kBBytes;
+      unsigned char* lo_t = hi_t + kBBytes;
+      for (int idx = t; idx < NB * 8; idx += 128) {
+        const int n = idx >> 3, c = idx & 7;
+        float v[8];
+        if (b0 + n < p.batch) {
+          const float4* src = reinterpret_cast<const float4*>(p.o + (size_t)(b0 + n) * p.K + kc * kTcK + c * 8);
+          const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+          v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+          v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = 0.f;
+        }
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * j]), h1 = __float2bfloat16_rn(v[2 * j + 1]);
+          const __nv_bfloat16 l0 = __float2bfloat16_rn(v[2 * j] - __bfloat162float(h0));
+          const __nv_bfloat16 l1 = __float2bfloat16_rn(v[2 * j + 1] - __bfloat162float(h1));
+          hw[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          lw[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+        }
+        const int off = n * 128 + ((c ^ (n & 7)) << 4);
+        *reinterpret_cast<uint4*>(hi_t + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(lo_t + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bfull[s]);
+    }
+  }
+
+  // accumulator complete
+  if (nst > 0 && !mbar_wait_bounded(done, 0)) ok = false;
+  if (!ok) {
+    s_fail = 1;
+    set_err(p.err, BASISKV_DEVERR_TIMEOUT);
+  }
+  tc_fence_after();
+  __syncthreads();  // every TMA landed and every MMA done: the A ring is free for `red`
+  fence_proxy_async_smem();
+  if (warp >= 1) {
+    const int q = warp & 3;
+    const int m = q * 32 + lane;
+#pragma unroll
+    for (int cc = 0; cc < NB; cc += 16) {
+      float v[16];
+      tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cc, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) red[m * NB + cc + j] = (nst > 0) ? v[j] : 0.f;
+    }
+  }
+  tc_fence_before();
+  cluster_sync();
+
+  // each CTA of the cluster sums its slice of rows over the cluster, in rank order
+  const int rows = kTcM / p.ksplit;
+  const int r0 = (int)rank * rows;
+  for (int idx = threadIdx.x; idx < rows * NB; idx += blockDim.x) {
+    const int n = idx / rows, m = r0 + idx % rows;
+    float acc = 0.f;
+    for (int q = 0; q < p.ksplit; ++q) acc += ld_dsmem_f32(red + m * NB + n, (uint32_t)q);
+    if (s_fail) acc = __int_as_float(0x7fc00000);  // NaN marks a result that cannot be trusted
+    if (b0 + n < p.batch) p.y[(size_t)(b0 + n) * p.hidden + c0 + m] = acc;
+  }
+  cluster_sync();  // no CTA leaves while its shared memory may still be read
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor map (cached per pointer/shape/device) and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+static cudaError_t gt_tensor_map(const void* Gt, int K, int hidden, CUtensorMap* out) {
+  struct Key {
+    int dev;
+    const void* ptr;
+    int K, hidden;
+    bool operator<(const Key& o) const {
+      return std::tie(dev, ptr, K, hidden) < std::tie(o.dev, o.ptr, o.K, o.hidden);
+    }
+  };
+  static std::mutex mu;
+  static std::map<Key, CUtensorMap> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const Key key{dev, Gt, K, hidden};
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return cudaSuccess;
+  }
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)hidden};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)kTcM};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Gt), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (cache.size() > 256) cache.clear();
+  cache[key] = map;
+  *out = map;
+  return cudaSuccess;
+}
+
+bool out_proj_tc_supported(int K, int hidden, int batch) {
+  return K % kTcK == 0 && hidden % kTcM == 0 && batch >= 1 && encode_fn() != nullptr;
+}
+
+static size_t tc_smem_bytes(int NB) {
+  return 1024 + (size_t)kTcStages * kTcABytes + (size_t)kTcStages * 2 * NB * kTcK * 2 + (3 * kTcStages + 1) * 8 + 16;
+}
+
+template <int NB>
+static cudaError_t launch_tc_nb(const CUtensorMap& map, OutProjTcParams p, int num_sms, cudaStream_t st) {
+  const int mtiles = p.hidden / kTcM;
+  const int bchunks = (p.batch + NB - 1) / NB;
+  const int KC = p.K / kTcK;
+  int ks = 1;
+  while (ks * 2 <= 8 && ks * 2 <= KC && (long long)mtiles * bchunks * ks * 2 <= num_sms) ks *= 2;
+  p.ksplit = ks;
+  p.chunks_per_cta = (KC + ks - 1) / ks;
+  const size_t smem = tc_smem_bytes(NB);
+  cudaError_t e = ensure_smem((const void*)out_proj_tc_kernel<NB>, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ks, mtiles, bchunks);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, out_proj_tc_kernel<NB>, map, p);
+}
+
+cudaError_t launch_out_proj_tc(const float* o, const void* Gt, float* y, int32_t* err, int batch, int K, int hidden,
+                               int num_sms, cudaStream_t st) {
+  CUtensorMap map;
+  cudaError_t e = gt_tensor_map(Gt, K, hidden, &map);
+  if (e != cudaSuccess) return e;
+  OutProjTcParams p{o, y, err, batch, K, hidden, 0, 1};
+  const int nb = batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 48 ? 48 : 64;
+  switch (nb) {
+    case 16: return launch_tc_nb<16>(map, p, num_sms, st);
+    case 32: return launch_tc_nb<32>(map, p, num_sms, st);
+    case 48: return launch_tc_nb<48>(map, p, num_sms, st);
+    default: return launch_tc_nb<64>(map, p, num_sms, st);
+  }
+}
+
+}  // namespace bkv
