@@ -156,6 +156,10 @@ BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basis
  * ascending order, padded with -1; sel_cnt [batch][Hq] int32.
  * scores (device, optional, may be NULL): [batch][Hq][max_pages] fp32, the
  * score of every page p < n_b (others untouched).
+ * With scores == NULL the call reads no summary of page 0 or of page n_b - 1
+ * (both are kept whatever they score), so it does not depend on
+ * basiskv_append of the same step, which only rewrites the recent page: the
+ * two may run concurrently on different streams.
  * workspace (device): at least basiskv_workspace_bytes(cfg, batch, max_pages)
  * bytes; contents need no initialisation and are clobbered.
  */

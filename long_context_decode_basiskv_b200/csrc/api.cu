@@ -54,30 +54,19 @@ static int num_sms() {
 }
 
 struct Workspace {
-  size_t scores, uni, ucnt, part, total;
-  int umax, nsplit, pps;
+  size_t scores, decode, total;
+  DecodePlan plan;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// routing scores first, then the decode scratch of decode_plan()
 static Workspace layout(const basiskv_config* c, int batch, int max_pages) {
   Workspace w{};
-  const int G = c->num_q_heads / c->num_kv_heads;
-  long long um = (long long)G * (c->top_k + 2);
-  if (um > max_pages) um = max_pages;
-  w.umax = (int)um;
-  w.pps = attn_pages_per_split(c->page_size);
-  w.nsplit = attn_nsplit(w.umax, c->page_size);
-  size_t off = 0;
-  w.scores = off;
-  off += up256((size_t)batch * c->num_q_heads * max_pages * 4);
-  w.uni = off;
-  off += up256((size_t)batch * c->num_kv_heads * w.umax * 4);
-  w.ucnt = off;
-  off += up256((size_t)batch * c->num_kv_heads * 4);
-  w.part = off;
-  off += up256((size_t)batch * c->num_q_heads * w.nsplit * (c->rank_v + 2) * 4);
-  w.total = off;
+  w.plan = decode_plan(c->num_q_heads, c->num_kv_heads, c->page_size, c->rank_v, c->top_k, batch, max_pages);
+  w.scores = 0;
+  w.decode = up256((size_t)batch * c->num_q_heads * max_pages * 4);
+  w.total = w.decode + w.plan.bytes;
   return w;
 }
 
@@ -143,7 +132,7 @@ basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cac
   float* sc = scores ? scores : reinterpret_cast<float*>(static_cast<char*>(ws) + w.scores);
   ScoreParams sp{q, cache->summary, cache->block_table, cache->seq_len, sc, err_flag,
                  batch, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cache->max_pages,
-                 cache->num_phys_pages, (cache->max_pages + 7) / 8};
+                 cache->num_phys_pages, (cache->max_pages + 7) / 8, scores ? 1 : 0};
   SelectParams selp{sc, cache->seq_len, sel, sel_cnt, cfg->num_q_heads, cfg->page_size,
                     cache->max_pages, cfg->top_k};
   return cuda_status(launch_route(sp, selp, cfg->head_dim, cfg->num_q_heads / cfg->num_kv_heads,
@@ -162,19 +151,10 @@ basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cach
   if (!aligned16(q)) return BASISKV_ERR_INVALID_ARG;
   const Workspace w = layout(cfg, batch, cache->max_pages);
   if (!ws || ws_bytes < w.total || !aligned16(ws)) return BASISKV_ERR_WORKSPACE;
-  char* base = static_cast<char*>(ws);
-  int32_t* uni = reinterpret_cast<int32_t*>(base + w.uni);
-  int32_t* ucnt = reinterpret_cast<int32_t*>(base + w.ucnt);
-  float* part = reinterpret_cast<float*>(base + w.part);
-  UnionParams up{sel, sel_cnt, cache->seq_len, uni, ucnt, err_flag, cfg->num_q_heads,
-                 cfg->num_kv_heads, cfg->page_size, cache->max_pages, cfg->top_k, w.umax};
-  AttnParams ap{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, uni, ucnt, part,
-                err_flag, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v,
-                cache->max_pages, cache->num_phys_pages, w.umax, w.pps, w.nsplit,
-                (float)(1.4426950408889634 / sqrt((double)cfg->head_dim)), 0};
-  CombineParams cp{part, ucnt, o_lat, cfg->num_q_heads, cfg->num_kv_heads, cfg->rank_v, w.pps, w.nsplit};
-  return cuda_status(launch_decode_attn(up, ap, cp, batch, cfg->head_dim, cfg->dtype == BASISKV_BF16,
-                                        (cudaStream_t)stream));
+  DecodeArgs a{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, sel, sel_cnt, o_lat, err_flag,
+               cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->page_size, cfg->rank_v,
+               cache->max_pages, cache->num_phys_pages, cfg->top_k, cfg->dtype == BASISKV_BF16};
+  return cuda_status(launch_decode_attn(w.plan, a, static_cast<char*>(ws) + w.decode, batch, (cudaStream_t)stream));
 }
 
 basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors* f, const float* o_lat,

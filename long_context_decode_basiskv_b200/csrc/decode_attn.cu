@@ -7,55 +7,93 @@
 // restricted to the selected tokens, with the weights applied to the rank-r
 // Value latents instead of full-width values.
 //
-// Three launches:
-//  union    one CTA per (sequence, KV head): merges the G query heads'
-//           selections into one ascending page list with a G-bit head mask
-//           per page, so a page chosen by several heads of a group is read once.
-//  attn     one CTA per (sequence, KV head, split of the union).  Each of its
-//           warps streams its own 16-token tiles (raw K rows and C rows,
-//           contiguous in the page block) through a private ring of shared
-//           memory stages filled by 1-D bulk copies (cp.async.bulk, mbarrier
-//           completion, no multicast).  Per tile and per head in the mask it
-//           forms 16 exact scores, updates an online softmax (running max and
-//           sum, base 2) and accumulates p * C.  Warps then merge in shared
-//           memory and the CTA writes one partial (max, sum, acc[r]) per head.
-//  combine  one CTA per (sequence, query head): log-sum-exp merge of the splits.
+// Two launches:
+//  union  one CTA per (sequence, KV head): merges the G query heads'
+//         selections into one ascending page list with a G-bit head mask per
+//         page (a page chosen by several heads of a group is read once), and
+//         zeroes the group's split counter.
+//  attn   one CTA per (sequence, KV head, split of the union).  Warp 0 is the
+//         producer: its lanes hold the split's union entries (page, mask,
+//         physical page, valid tokens) and lane 0 streams 16-token tiles (raw
+//         K rows and C rows, each contiguous in the page block) into a ring of
+//         shared-memory stages with 1-D bulk copies (cp.async.bulk, mbarrier
+//         completion, no multicast), writing each stage's head mask beside it.
+//         Warps 1..G are the consumers, one per query head of the group: a warp
+//         whose head selected the tile forms its 16 exact scores, updates an
+//         online softmax (running max and sum, base 2) and accumulates p * C;
+//         every consumer releases the stage.  Each head's split result (max,
+//         sum, acc[r]) goes to the workspace; the last CTA of a group to finish
+//         (counted with an atomic) merges the group's splits with the
+//         log-sum-exp rule and writes o_lat.
 // HBM-bound: every byte of the union's pages is read once.
 #include "kernels.cuh"
 
 namespace bkv {
 
-constexpr int kTile = 16;          // tokens per tile
-constexpr int kAttnWarps = 4;      // warps per CTA
-constexpr int kMaxStages = 4;      // ring depth per warp (fewer when shared memory is short)
-constexpr int kTilesPerSplit = 32; // tiles of union pages handled by one CTA
+constexpr int kTile = 16;           // tokens per tile
+constexpr int kStages = 4;          // ring depth per CTA
+constexpr int kTargetCtas = 888;    // one wave of attn CTAs on a B200 (148 SMs x 6)
+
+// ---------------------------------------------------------------------------
+// plan: tiles per split and scratch layout (independent of the device)
+// ---------------------------------------------------------------------------
+static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages) {
+  DecodePlan pl{};
+  const int G = Hq / Hkv;
+  long long um = (long long)G * (top_k + 2);
+  if (um > max_pages) um = max_pages;
+  pl.umax = (int)um;
+  pl.tpp = page / kTile;
+  const long long groups = (long long)batch * Hkv;
+  const long long tiles = (long long)pl.umax * pl.tpp;
+  long long eps = (tiles * groups + kTargetCtas - 1) / kTargetCtas;  // tiles per split, then pages
+  eps = (eps + pl.tpp - 1) / pl.tpp;
+  if (eps < 1) eps = 1;
+  pl.eps = (int)eps;
+  pl.nsplit = (pl.umax + pl.eps - 1) / pl.eps;
+  size_t off = 0;
+  pl.uni_off = off;
+  off += up256((size_t)batch * Hkv * pl.umax * 4);
+  pl.ucnt_off = off;
+  off += up256((size_t)batch * Hkv * 4);
+  pl.cnt_off = off;
+  off += up256((size_t)batch * Hkv * 4);
+  pl.part_off = off;
+  off += up256((size_t)batch * Hq * pl.nsplit * (r + 2) * 4);
+  pl.bytes = off;
+  return pl;
+}
 
 // ---------------------------------------------------------------------------
 // union of the group's selections
 // ---------------------------------------------------------------------------
-
-
 __global__ void __launch_bounds__(256) union_kernel(UnionParams p) {
   extern __shared__ __align__(16) uint32_t words[];  // [ceil(max_pages / 4)] byte masks
   __shared__ int warp_tot[32];
+  __shared__ int s_cnt[8];
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int G = p.Hq / p.Hkv;
+  const int row_len = p.top_k + 2;
+  const size_t row0 = (size_t)b * p.Hq + (size_t)g * G;
   const int L = p.seq_len[b];
   const int n = min((L + p.page - 1) / p.page, p.max_pages);
   const int nw = (n + 3) / 4;
+  if (tid == 0) p.cnt[(size_t)b * p.Hkv + g] = 0;
+  if (tid < G) s_cnt[tid] = min(p.sel_cnt[row0 + tid], row_len);
   for (int i = tid; i < nw; i += blockDim.x) words[i] = 0u;
   __syncthreads();
-  for (int hi = 0; hi < G; ++hi) {
-    const size_t row = (size_t)b * p.Hq + g * G + hi;
-    const int cnt = min(p.sel_cnt[row], p.top_k + 2);
-    for (int i = tid; i < cnt; i += blockDim.x) {
-      const int pg = p.sel[row * (p.top_k + 2) + i];
-      if (pg < 0 || pg >= n) {
-        set_err(p.err, BASISKV_DEVERR_SELECTION);
-        continue;
-      }
-      atomicOr(&words[pg >> 2], (1u << hi) << ((pg & 3) * 8));
+  // the G selection rows are contiguous: one flat pass, every load issued at once
+  for (int i = tid; i < G * row_len; i += blockDim.x) {
+    const int hi = i / row_len;
+    if (i - hi * row_len >= s_cnt[hi]) continue;
+    const int pg = p.sel[row0 * row_len + i];
+    if (pg < 0 || pg >= n) {
+      set_err(p.err, BASISKV_DEVERR_SELECTION);
+      continue;
     }
+    atomicOr(&words[pg >> 2], (1u << hi) << ((pg & 3) * 8));
   }
   __syncthreads();
   const int per = (n + blockDim.x - 1) / blockDim.x;
@@ -79,15 +117,13 @@ __global__ void __launch_bounds__(256) union_kernel(UnionParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// split attention
+// split attention with in-kernel merge
 // ---------------------------------------------------------------------------
-
-
 template <typename T, int D>
-struct TileLoad {
+struct KRow {
   static constexpr int DPL = D / 32;
-  // lane's DPL consecutive elements of row j
-  static __device__ __forceinline__ void row(const T* tile, int j, int lane, float (&out)[DPL]) {
+  // lane's DPL consecutive elements of row j of a [16][D] tile
+  static __device__ __forceinline__ void load(const T* tile, int j, int lane, float (&out)[DPL]) {
     const T* src = tile + j * D + lane * DPL;
     if constexpr (sizeof(T) == 2 && DPL == 4) {
       const uint2 w = *reinterpret_cast<const uint2*>(src);
@@ -105,291 +141,253 @@ struct TileLoad {
   }
 };
 
-template <typename T, int D, int G, int RPL>
-__global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(AttnParams p) {
+// two consecutive latent dims (dim, dim + 1) of one C row
+template <typename T>
+__device__ __forceinline__ void load_pair(const T* row, int dim, float& a, float& b) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + dim);
+    a = bf16lo(w);
+    b = bf16hi(w);
+  } else {
+    const float2 w = *reinterpret_cast<const float2*>(row + dim);
+    a = w.x;
+    b = w.y;
+  }
+}
+
+template <typename T, int D, int G, int CU>
+__global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   constexpr int DPL = D / 32;
   extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ uint32_t meta[kStages];  // head mask | valid tokens << 8 of the tile in each stage
+  __shared__ int s_last;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.r;
-  const int U = p.ucnt[(size_t)b * p.Hkv + g];
-  const int e0 = split * p.pps;
-  if (e0 >= U) return;  // whole CTA idle (uniform)
-  const int e1 = min(U, e0 + p.pps);
-  const int L = p.seq_len[b];
-  const int n = min((L + p.page - 1) / p.page, p.max_pages);  // union entries are < n
-  const int last_valid = L - (n - 1) * p.page;
-  const int tpp = p.page / kTile;
-  const int ntiles = (e1 - e0) * tpp;
+  const size_t bg = (size_t)b * p.Hkv + g;
+  const int U = p.ucnt[bg];
+  const int e0 = split * p.eps;
+  const int nsplit_active = (U + p.eps - 1) / p.eps;
+  if (e0 >= U) {
+    // no work in this split; split 0 of an empty group still defines its output
+    if (split == 0 && U == 0)
+      for (int i = threadIdx.x; i < G * r; i += blockDim.x)
+        p.o_lat[((size_t)b * p.Hq + (size_t)g * G) * r + i] = 0.f;
+    return;
+  }
+  const int nent = min(U, e0 + p.eps) - e0;
+  const int ntiles = nent * p.tpp;
 
   const uint32_t k_bytes = kTile * D * sizeof(T);
   const uint32_t c_bytes = kTile * r * sizeof(T);
   const uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
-  const int kStages = p.nstages;
-  unsigned char* ring = smem + (size_t)w * kStages * stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kAttnWarps * kStages * stage_bytes) + w * kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * stage_bytes);
+  uint64_t* empty = full + kStages;
 
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], G);
+    }
     fence_mbar_init();
   }
-  __syncwarp();
-
-  const int32_t* uni = p.uni + ((size_t)b * p.Hkv + g) * p.umax;
-  const T* kbase = static_cast<const T*>(p.k_raw);
-  const T* cbase = static_cast<const T*>(p.c_lat);
-
-  // tile t of this split -> source pointers, valid tokens, head mask
-  auto desc = [&](int t, const T*& kp, const T*& cp, int& valid, uint32_t& mask) {
-    const int e = e0 + t / tpp, sub = t - (t / tpp) * tpp;
-    const uint32_t ent = (uint32_t)uni[e];
-    const int pg = (int)(ent & 0xffffffu);
-    mask = ent >> 24;
-    valid = (pg == n - 1) ? min(kTile, max(0, last_valid - sub * kTile)) : kTile;
-    kp = nullptr;
-    cp = nullptr;
-    if (pg >= n) {
-      valid = 0;
-      return;
-    }
-    const int phys = p.block_table[(size_t)b * p.max_pages + pg];
-    if (phys < 0 || phys >= p.num_phys) {
-      valid = 0;
-      if (lane == 0) set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
-      return;
-    }
-    const size_t row0 = ((size_t)phys * p.Hkv + g) * p.page + (size_t)sub * kTile;
-    kp = kbase + row0 * D;
-    cp = cbase + row0 * r;
-  };
-
-  auto issue = [&](int i) {  // i-th tile of this warp into stage i % kStages
-    const T* kp;
-    const T* cp;
-    int valid;
-    uint32_t mask;
-    desc(w + i * kAttnWarps, kp, cp, valid, mask);
-    if (lane == 0) {
-      uint64_t* bar = &bars[i % kStages];
-      unsigned char* st = ring + (size_t)(i % kStages) * stage_bytes;
-      fence_proxy_async_smem();
-      if (valid > 0) {
-        mbar_arrive_expect_tx(bar, k_bytes + c_bytes);
-        bulk_g2s(st, kp, k_bytes, bar);
-        bulk_g2s(st + k_bytes, cp, c_bytes, bar);
-      } else {
-        mbar_arrive_expect_tx(bar, 0);
-      }
-    }
-  };
-
-  // per-head query (pre-scaled for base-2 softmax) and running state
-  float qf[G][DPL];
-  {
-    const T* qb = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
-#pragma unroll
-    for (int hi = 0; hi < G; ++hi)
-#pragma unroll
-      for (int u = 0; u < DPL; ++u) qf[hi][u] = Elem<T>::to_f(qb[hi * D + lane * DPL + u]) * p.qscale;
-  }
-  float m_run[G], l_run[G], acc[G][RPL];
-#pragma unroll
-  for (int hi = 0; hi < G; ++hi) {
-    m_run[hi] = -INFINITY;
-    l_run[hi] = 0.f;
-#pragma unroll
-    for (int u = 0; u < RPL; ++u) acc[hi][u] = 0.f;
-  }
-
-  const int my_count = (ntiles > w) ? (ntiles - w + kAttnWarps - 1) / kAttnWarps : 0;
-  const int pre = min(kStages, my_count);
-  for (int i = 0; i < pre; ++i) issue(i);
+  __syncthreads();
 
   bool ok = true;
-  for (int i = 0; i < my_count; ++i) {
-    const int st_idx = i % kStages;
-    const uint32_t parity = (uint32_t)((i / kStages) & 1);
-    if (!mbar_wait_bounded(&bars[st_idx], parity)) {
-      if (lane == 0) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
-      // let the copies already in flight land before the CTA leaves
-      for (int j = i + 1; j < min(my_count, i + kStages); ++j)
-        mbar_wait_bounded(&bars[j % kStages], (uint32_t)((j / kStages) & 1), 200000000LL);
-      ok = false;
-      break;
-    }
-    const T* kp;
-    const T* cp;
-    int valid;
-    uint32_t mask;
-    desc(w + i * kAttnWarps, kp, cp, valid, mask);
-    if (valid > 0) {
-      const T* ks = reinterpret_cast<const T*>(ring + (size_t)st_idx * stage_bytes);
-      const T* cs = reinterpret_cast<const T*>(ring + (size_t)st_idx * stage_bytes + k_bytes);
-      float kf[kTile][DPL];
-#pragma unroll
-      for (int j = 0; j < kTile; ++j) TileLoad<T, D>::row(ks, j, lane, kf[j]);
-      // latents of slots past the valid tokens of a partial page are never
-      // written: zero them so that 0 * (stale bits) cannot inject NaN
-      float cf[kTile][RPL];
-#pragma unroll
-      for (int j = 0; j < kTile; ++j)
-#pragma unroll
-        for (int u = 0; u < RPL; ++u) {
-          const int dim = u * 32 + lane;
-          cf[j][u] = (dim < r && j < valid) ? Elem<T>::to_f(cs[j * r + dim]) : 0.f;
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    const int L = p.seq_len[b];
+    const int n = min((L + p.page - 1) / p.page, p.max_pages);
+    const int last_valid = L - (n - 1) * p.page;
+    const int32_t* uni = p.uni + bg * p.umax;
+    const T* kbase = static_cast<const T*>(p.k_raw);
+    const T* cbase = static_cast<const T*>(p.c_lat);
+    for (int cb = 0; cb < nent && ok; cb += 32) {
+      // lane e holds union entry e0 + cb + e
+      uint32_t my_mask = 0;
+      int my_phys = -1, my_valid = 0;
+      if (cb + lane < nent) {
+        const uint32_t ent = (uint32_t)uni[e0 + cb + lane];
+        const int pg = (int)(ent & 0xffffffu);
+        my_mask = ent >> 24;
+        if (pg < n) {
+          const int ph = p.block_table[(size_t)b * p.max_pages + pg];
+          if (ph >= 0 && ph < p.num_phys) {
+            my_phys = ph;
+            my_valid = (pg == n - 1) ? last_valid : p.page;
+          } else {
+            set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
+          }
         }
-      const bool tok_ok = (lane >> 1) < valid;
+      }
+      const int t_end = min(nent, cb + 32) * p.tpp;
+      for (int t = cb * p.tpp; t < t_end; ++t) {
+        const int el = t / p.tpp - cb, sub = t - (t / p.tpp) * p.tpp;
+        const int ph = __shfl_sync(kFull, my_phys, el);
+        const uint32_t mask = __shfl_sync(kFull, my_mask, el);
+        const int pv = __shfl_sync(kFull, my_valid, el);
+        const int valid = (ph >= 0) ? min(kTile, max(0, pv - sub * kTile)) : 0;
+        const int s = t % kStages;
+        if (t >= kStages && !mbar_wait_bounded(&empty[s], (uint32_t)(((t / kStages) - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          meta[s] = mask | ((uint32_t)valid << 8);
+          unsigned char* st = smem + (size_t)s * stage_bytes;
+          fence_proxy_async_smem();
+          if (valid > 0) {
+            const size_t row0 = ((size_t)ph * p.Hkv + g) * p.page + (size_t)sub * kTile;
+            mbar_arrive_expect_tx(&full[s], k_bytes + c_bytes);
+            bulk_g2s(st, kbase + row0 * D, k_bytes, &full[s]);
+            bulk_g2s(st + k_bytes, cbase + row0 * r, c_bytes, &full[s]);
+          } else {
+            mbar_arrive_expect_tx(&full[s], 0);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else {
+    // ---------------- consumer: one query head ----------------
+    const int hi = warp - 1;
+    const int h = g * G + hi;
+    float qf[DPL];
+    {
+      const T* qr = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D + lane * DPL;
 #pragma unroll
-      for (int hi = 0; hi < G; ++hi) {
-        if (!((mask >> hi) & 1u)) continue;  // warp-uniform
-        float s[kTile];
+      for (int u = 0; u < DPL; ++u) qf[u] = Elem<T>::to_f(qr[u]) * p.qscale;
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    float acc[CU][2];
+#pragma unroll
+    for (int u = 0; u < CU; ++u) acc[u][0] = acc[u][1] = 0.f;
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kStages;
+      if (!mbar_wait_bounded(&full[s], (uint32_t)((t / kStages) & 1))) {
+        ok = false;
+        break;
+      }
+      const uint32_t mt = meta[s];
+      const int valid = (int)(mt >> 8);
+      if (((mt >> hi) & 1u) && valid > 0) {
+        const T* ks = reinterpret_cast<const T*>(smem + (size_t)s * stage_bytes);
+        const T* cs = reinterpret_cast<const T*>(smem + (size_t)s * stage_bytes + k_bytes);
+        float sc[kTile];
 #pragma unroll
         for (int j = 0; j < kTile; ++j) {
+          float kv[DPL];
+          KRow<T, D>::load(ks, j, lane, kv);
           float a = 0.f;
 #pragma unroll
-          for (int u = 0; u < DPL; ++u) a = fmaf(qf[hi][u], kf[j][u], a);
-          s[j] = a;
+          for (int u = 0; u < DPL; ++u) a = fmaf(qf[u], kv[u], a);
+          sc[j] = a;
         }
-        transpose_reduce<kTile>(s, lane);  // lane holds token (lane >> 1)
-        const float sj = tok_ok ? s[0] : -INFINITY;
+        transpose_reduce<kTile>(sc, lane);  // lane holds token (lane >> 1)
+        const float sj = ((lane >> 1) < valid) ? sc[0] : -INFINITY;
         float mx = sj;
 #pragma unroll
         for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-        const float m_new = fmaxf(m_run[hi], mx);
-        const float corr = exp2f(m_run[hi] - m_new);
+        const float m_new = fmaxf(m_run, mx);
+        const float corr = exp2f(m_run - m_new);
         const float pj = exp2f(sj - m_new);
-        l_run[hi] = l_run[hi] * corr + ((lane & 1) ? 0.f : pj);
+        l_run = l_run * corr + ((lane & 1) ? 0.f : pj);
 #pragma unroll
-        for (int u = 0; u < RPL; ++u) acc[hi][u] *= corr;
+        for (int u = 0; u < CU; ++u) {
+          acc[u][0] *= corr;
+          acc[u][1] *= corr;
+        }
 #pragma unroll
         for (int j = 0; j < kTile; ++j) {
           const float pb = __shfl_sync(kFull, pj, 2 * j);
+          if (j < valid) {  // slots past the valid tokens hold stale bits
 #pragma unroll
-          for (int u = 0; u < RPL; ++u) acc[hi][u] = fmaf(pb, cf[j][u], acc[hi][u]);
+            for (int u = 0; u < CU; ++u) {
+              const int dim = 64 * u + 2 * lane;
+              if (dim < r) {
+                float c0, c1;
+                load_pair<T>(cs + j * r, dim, c0, c1);
+                acc[u][0] = fmaf(pb, c0, acc[u][0]);
+                acc[u][1] = fmaf(pb, c1, acc[u][1]);
+              }
+            }
+          }
         }
-        m_run[hi] = m_new;
+        m_run = m_new;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-    __syncwarp();
-    if (i + kStages < my_count) issue(i + kStages);
-  }
-  (void)ok;
-
-  // merge the warps of this CTA, write one partial per head
-  __syncthreads();
-  const int stride = 2 + RPL * 32;
-  float* mb = reinterpret_cast<float*>(smem);  // [warps][G][stride]
-#pragma unroll
-  for (int hi = 0; hi < G; ++hi) {
-    const float lsum = warp_sum(l_run[hi]);
-    float* dst = mb + ((size_t)w * G + hi) * stride;
+    // this head's result for the split
+    const float lsum = warp_sum(l_run);
+    float* out = p.part + (((size_t)b * p.Hq + h) * p.nsplit + split) * (r + 2);
     if (lane == 0) {
-      dst[0] = m_run[hi];
-      dst[1] = lsum;
+      out[0] = m_run;
+      out[1] = lsum;
     }
 #pragma unroll
-    for (int u = 0; u < RPL; ++u) dst[2 + u * 32 + lane] = acc[hi][u];
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < G * r; idx += blockDim.x) {
-    const int hi = idx / r, dim = idx - hi * r;
-    float M = -INFINITY;
-#pragma unroll
-    for (int ww = 0; ww < kAttnWarps; ++ww) M = fmaxf(M, mb[((size_t)ww * G + hi) * stride]);
-    float Ls = 0.f, As = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int ww = 0; ww < kAttnWarps; ++ww) {
-        const float* src = mb + ((size_t)ww * G + hi) * stride;
-        const float f = exp2f(src[0] - M);  // 0 for a warp that saw nothing of this head
-        Ls += src[1] * f;
-        As += src[2 + dim] * f;
+    for (int u = 0; u < CU; ++u) {
+      const int dim = 64 * u + 2 * lane;
+      if (dim < r) {
+        out[2 + dim] = acc[u][0];
+        out[3 + dim] = acc[u][1];
       }
     }
-    float* out = p.part + (((size_t)b * p.Hq + (size_t)g * G + hi) * p.nsplit + split) * (r + 2);
-    out[2 + dim] = As;
-    if (dim == 0) {
-      out[0] = M;
-      out[1] = Ls;
-    }
   }
-}
+  if (!ok) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
 
-// ---------------------------------------------------------------------------
-// combine splits
-// ---------------------------------------------------------------------------
-
-
-__global__ void __launch_bounds__(128) combine_kernel(CombineParams p) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int G = p.Hq / p.Hkv;
-  const int U = p.ucnt[(size_t)b * p.Hkv + h / G];
-  const int ns = min(p.nsplit, (U + p.pps - 1) / p.pps);
-  const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * (p.r + 2);
+  // the last CTA of the group to finish merges every split of its G heads
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[bg], 1) == nsplit_active - 1);
+  __syncthreads();
+  if (!s_last || warp == 0) return;
+  __threadfence();
+  const int hi = warp - 1;
+  const int h = g * G + hi;
+  const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * (r + 2);
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, base[(size_t)s * (p.r + 2)]);
+  for (int s = lane; s < nsplit_active; s += 32) M = fmaxf(M, __ldcg(base + (size_t)s * (r + 2)));
+  M = warp_max(M);
   float Ls = 0.f;
-  if (M != -INFINITY)
-    for (int s = 0; s < ns; ++s) {
-      const float* ps = base + (size_t)s * (p.r + 2);
-      Ls += ps[1] * exp2f(ps[0] - M);
-    }
-  for (int dim = threadIdx.x; dim < p.r; dim += blockDim.x) {
+  for (int s = lane; s < nsplit_active; s += 32) {
+    const float ms = __ldcg(base + (size_t)s * (r + 2));
+    if (ms != -INFINITY) Ls += __ldcg(base + (size_t)s * (r + 2) + 1) * exp2f(ms - M);
+  }
+  Ls = warp_sum(Ls);
+  for (int dim = lane; dim < r; dim += 32) {
     float a = 0.f;
     if (M != -INFINITY)
-      for (int s = 0; s < ns; ++s) {
-        const float* ps = base + (size_t)s * (p.r + 2);
-        a += ps[2 + dim] * exp2f(ps[0] - M);
+      for (int s = 0; s < nsplit_active; ++s) {
+        const float* ps = base + (size_t)s * (r + 2);
+        const float ms = __ldcg(ps);
+        if (ms != -INFINITY) a += __ldcg(ps + 2 + dim) * exp2f(ms - M);
       }
-    p.o_lat[((size_t)b * p.Hq + h) * p.r + dim] = (Ls > 0.f) ? a / Ls : 0.f;
+    p.o_lat[((size_t)b * p.Hq + h) * r + dim] = (Ls > 0.f) ? a / Ls : 0.f;
   }
 }
 
 // ---------------------------------------------------------------------------
 // launch
 // ---------------------------------------------------------------------------
-int attn_pages_per_split(int page) { return max(1, kTilesPerSplit / (page / kTile)); }
-int attn_nsplit(int umax, int page) {
-  const int pps = attn_pages_per_split(page);
-  return (umax + pps - 1) / pps;
-}
-constexpr size_t kSmemLimit = 227 * 1024;
-
-int attn_stages(int d, int r, int esize) {
+size_t attn_smem_bytes(int d, int r, int esize) {
   const size_t stage = ((size_t)kTile * (d + r) * esize + 127) & ~(size_t)127;
-  int n = kMaxStages;
-  while (n > 1 && (size_t)kAttnWarps * n * (stage + 8) > kSmemLimit) --n;
-  return n;
+  return (size_t)kStages * stage + 2 * kStages * 8;
 }
 
-size_t attn_smem_bytes(int d, int r, int esize, int G, int rpl, int nstages) {
-  const size_t stage = ((size_t)kTile * (d + r) * esize + 127) & ~(size_t)127;
-  size_t ring = (size_t)kAttnWarps * nstages * stage + (size_t)kAttnWarps * nstages * 8;
-  const size_t merge = (size_t)kAttnWarps * G * (2 + rpl * 32) * 4;
-  return ring > merge ? ring : merge;
-}
-
-template <typename T, int D, int G, int RPL>
+template <typename T, int D, int G, int CU>
 static cudaError_t launch_attn_t(const AttnParams& p, int batch, cudaStream_t st) {
-  const size_t smem = attn_smem_bytes(D, p.r, sizeof(T), G, RPL, p.nstages);
-  cudaError_t e = ensure_smem((const void*)attn_kernel<T, D, G, RPL>, smem);
+  const size_t smem = attn_smem_bytes(D, p.r, sizeof(T));
+  cudaError_t e = ensure_smem((const void*)attn_kernel<T, D, G, CU>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nsplit, p.Hkv, batch);
-  attn_kernel<T, D, G, RPL><<<grid, kAttnWarps * 32, smem, st>>>(p);
+  attn_kernel<T, D, G, CU><<<grid, 32 * (G + 1), smem, st>>>(p);
   return cudaGetLastError();
 }
 
 template <typename T, int D, int G>
-static cudaError_t launch_attn_r(AttnParams p, int batch, cudaStream_t st) {
-  p.nstages = attn_stages(D, p.r, sizeof(T));
-  const int rpl = (p.r + 31) / 32;
-  switch (rpl) {
-    case 1: return launch_attn_t<T, D, G, 1>(p, batch, st);
-    case 2: return launch_attn_t<T, D, G, 2>(p, batch, st);
-    case 3: return launch_attn_t<T, D, G, 3>(p, batch, st);
-    case 4: return launch_attn_t<T, D, G, 4>(p, batch, st);
-    default: return cudaErrorInvalidValue;
-  }
+static cudaError_t launch_attn_r(const AttnParams& p, int batch, cudaStream_t st) {
+  return (p.r <= 64) ? launch_attn_t<T, D, G, 1>(p, batch, st) : launch_attn_t<T, D, G, 2>(p, batch, st);
 }
 
 template <typename T, int D>
@@ -403,24 +401,28 @@ static cudaError_t launch_attn_g(const AttnParams& p, int G, int batch, cudaStre
   }
 }
 
-cudaError_t launch_decode_attn(const UnionParams& up, const AttnParams& ap, const CombineParams& cp,
-                               int batch, int d, bool bf16, cudaStream_t st) {
-  const size_t usmem = ((size_t)up.max_pages + 3) / 4 * 4;
-  cudaError_t e0 = ensure_smem((const void*)union_kernel, usmem);
-  if (e0 != cudaSuccess) return e0;
-  union_kernel<<<dim3(up.Hkv, batch), 256, usmem, st>>>(up);
-  cudaError_t e = cudaGetLastError();
+cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* scratch, int batch,
+                               cudaStream_t st) {
+  char* base = static_cast<char*>(scratch);
+  int32_t* uni = reinterpret_cast<int32_t*>(base + pl.uni_off);
+  int32_t* ucnt = reinterpret_cast<int32_t*>(base + pl.ucnt_off);
+  int32_t* cnt = reinterpret_cast<int32_t*>(base + pl.cnt_off);
+  float* part = reinterpret_cast<float*>(base + pl.part_off);
+  UnionParams up{a.sel, a.sel_cnt, a.seq_len, uni, ucnt, cnt, a.err, a.Hq, a.Hkv, a.page, a.max_pages, a.top_k,
+                 pl.umax};
+  const size_t usmem = ((size_t)a.max_pages + 3) / 4 * 4;
+  cudaError_t e = ensure_smem((const void*)union_kernel, usmem);
   if (e != cudaSuccess) return e;
-  const int G = ap.Hq / ap.Hkv;
-  if (bf16)
-    e = (d == 128) ? launch_attn_g<__nv_bfloat16, 128>(ap, G, batch, st)
-                   : launch_attn_g<__nv_bfloat16, 64>(ap, G, batch, st);
-  else
-    e = (d == 128) ? launch_attn_g<float, 128>(ap, G, batch, st)
-                   : launch_attn_g<float, 64>(ap, G, batch, st);
-  if (e != cudaSuccess) return e;
-  combine_kernel<<<dim3(cp.Hq, batch), 128, 0, st>>>(cp);
-  return cudaGetLastError();
+  union_kernel<<<dim3(a.Hkv, batch), 256, usmem, st>>>(up);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  AttnParams ap{a.q, a.k_raw, a.c_lat, a.block_table, a.seq_len, uni, ucnt, cnt, part, a.o_lat, a.err,
+                a.Hq, a.Hkv, a.page, a.r, a.max_pages, a.num_phys, pl.umax, pl.tpp, pl.eps, pl.nsplit,
+                (float)(1.4426950408889634 / sqrt((double)a.d))};
+  const int G = a.Hq / a.Hkv;
+  if (a.bf16)
+    return (a.d == 128) ? launch_attn_g<__nv_bfloat16, 128>(ap, G, batch, st)
+                        : launch_attn_g<__nv_bfloat16, 64>(ap, G, batch, st);
+  return (a.d == 128) ? launch_attn_g<float, 128>(ap, G, batch, st) : launch_attn_g<float, 64>(ap, G, batch, st);
 }
 
 }  // namespace bkv

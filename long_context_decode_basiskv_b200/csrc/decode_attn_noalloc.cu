@@ -48,8 +48,6 @@ cudaError_t scratch_address(void** out) {
   return cudaSuccess;
 }
 
-size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
-
 }  // namespace
 }  // namespace bkv
 
@@ -65,22 +63,14 @@ extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
   if (batch == 0) return BASISKV_OK;
   if (cache->max_pages <= 0) return BASISKV_ERR_INVALID_ARG;
 
-  // the same scratch regions basiskv_decode_attn takes from its workspace
-  const int G = cfg->num_q_heads / cfg->num_kv_heads;
-  long long um = (long long)G * (cfg->top_k + 2);
-  if (um > cache->max_pages) um = cache->max_pages;
-  const int umax = (int)um;
-  const int pps = attn_pages_per_split(cfg->page_size);
-  const int nsplit = attn_nsplit(umax, cfg->page_size);
-  const size_t uni_off = 0;
-  const size_t ucnt_off = uni_off + up256((size_t)batch * cfg->num_kv_heads * umax * 4);
-  const size_t part_off = ucnt_off + up256((size_t)batch * cfg->num_kv_heads * 4);
-  const size_t need = part_off + up256((size_t)batch * cfg->num_q_heads * nsplit * (cfg->rank_v + 2) * 4);
-  if (need > kNoAllocScratchBytes) {
+  // the same scratch basiskv_decode_attn takes from its workspace
+  const DecodePlan plan = decode_plan(cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v, cfg->top_k,
+                                      batch, cache->max_pages);
+  if (plan.bytes > kNoAllocScratchBytes) {
     fprintf(stderr,
             "basiskv_decode_attn_noalloc: this shape needs %zu bytes of scratch, more than the "
             "fixed %zu; use basiskv_decode_attn with a workspace\n",
-            need, kNoAllocScratchBytes);
+            plan.bytes, kNoAllocScratchBytes);
     return BASISKV_ERR_WORKSPACE;
   }
 
@@ -102,19 +92,10 @@ extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
             cudaGetErrorString(e));
     return BASISKV_ERR_CUDA;
   }
-  char* base = static_cast<char*>(scratch);
-  int32_t* uni = reinterpret_cast<int32_t*>(base + uni_off);
-  int32_t* ucnt = reinterpret_cast<int32_t*>(base + ucnt_off);
-  float* part = reinterpret_cast<float*>(base + part_off);
-  UnionParams up{sel, sel_cnt, cache->seq_len, uni, ucnt, err_flag, cfg->num_q_heads,
-                 cfg->num_kv_heads, cfg->page_size, cache->max_pages, cfg->top_k, umax};
-  AttnParams ap{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, uni, ucnt, part,
-                err_flag, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v,
-                cache->max_pages, cache->num_phys_pages, umax, pps, nsplit,
-                (float)(1.4426950408889634 / sqrt((double)cfg->head_dim)), 0};
-  CombineParams cp{part, ucnt, o_lat, cfg->num_q_heads, cfg->num_kv_heads, cfg->rank_v, pps, nsplit};
-  e = launch_decode_attn(up, ap, cp, batch, cfg->head_dim, cfg->dtype == BASISKV_BF16,
-                         (cudaStream_t)stream);
+  DecodeArgs a{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, sel, sel_cnt, o_lat, err_flag,
+               cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->page_size, cfg->rank_v,
+               cache->max_pages, cache->num_phys_pages, cfg->top_k, cfg->dtype == BASISKV_BF16};
+  e = launch_decode_attn(plan, a, scratch, batch, (cudaStream_t)stream);
   if (e != cudaSuccess) {
     fprintf(stderr, "basiskv_decode_attn_noalloc: CUDA error %s\n", cudaGetErrorString(e));
     return BASISKV_ERR_CUDA;

@@ -31,6 +31,7 @@ struct ScoreParams {
   int32_t* err;
   int batch, Hq, Hkv, page, max_pages, num_phys;
   int page_batches;
+  int all_pages;  // 0: skip the sink and recent pages (always kept; their scores are not needed)
 };
 struct SelectParams {
   const float* scores;
@@ -46,8 +47,9 @@ struct UnionParams {
   const int32_t* sel;
   const int32_t* sel_cnt;
   const int32_t* seq_len;
-  int32_t* uni;
-  int32_t* ucnt;
+  int32_t* uni;   // [B][Hkv][umax]  page | head mask << 24
+  int32_t* ucnt;  // [B][Hkv]
+  int32_t* cnt;   // [B][Hkv] finished-split counters (zeroed here)
   int32_t* err;
   int Hq, Hkv, page, max_pages, top_k, umax;
 };
@@ -59,22 +61,40 @@ struct AttnParams {
   const int32_t* seq_len;
   const int32_t* uni;
   const int32_t* ucnt;
-  float* part;
+  int32_t* cnt;
+  float* part;   // [B][Hq][nsplit][r + 2]
+  float* o_lat;  // [B][Hq][r]
   int32_t* err;
-  int Hq, Hkv, page, r, max_pages, num_phys, umax, pps, nsplit;
-  float qscale;
-  int nstages;  // set by the launcher
+  int Hq, Hkv, page, r, max_pages, num_phys, umax, tpp, eps, nsplit;
+  float qscale;  // log2(e) / sqrt(d)
 };
-struct CombineParams {
-  const float* part;
-  const int32_t* ucnt;
+
+// Tiles per split and scratch layout of one decode_attn call; depends on the
+// shape only, so the workspace query and every launch agree on it.
+struct DecodePlan {
+  int umax;    // max union pages per (sequence, KV head)
+  int tpp;     // 16-token tiles per page
+  int eps;     // union pages per split
+  int nsplit;  // splits per (sequence, KV head)
+  size_t uni_off, ucnt_off, cnt_off, part_off, bytes;
+};
+DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages);
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_raw;
+  const void* c_lat;
+  const int32_t* block_table;
+  const int32_t* seq_len;
+  const int32_t* sel;
+  const int32_t* sel_cnt;
   float* o_lat;
-  int Hq, Hkv, r, pps, nsplit;
+  int32_t* err;
+  int Hq, Hkv, d, page, r, max_pages, num_phys, top_k;
+  bool bf16;
 };
-int attn_pages_per_split(int page);
-int attn_nsplit(int umax, int page);
-cudaError_t launch_decode_attn(const UnionParams& up, const AttnParams& ap, const CombineParams& cp,
-                               int batch, int d, bool bf16, cudaStream_t st);
+cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* scratch, int batch,
+                               cudaStream_t st);
 
 struct OutProjParams {
   const float* o;

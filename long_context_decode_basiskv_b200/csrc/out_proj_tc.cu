@@ -8,9 +8,11 @@
 // product keeps fp32-level accuracy with bf16 operands.
 //
 // Per CTA: warp 0 streams 128x64 tiles of Gt with 2-D TMA (128-byte swizzle,
-// no multicast) into a 4-stage ring and one of its threads issues the
-// tcgen05.mma instructions; warps 1-4 write the swizzled bf16 hi/lo tiles of
-// o into a matching ring and, at the end, read the accumulator out of TMEM.
+// no multicast) into a ring of 4-8 stages and one of its threads issues the
+// tcgen05.mma instructions, refilling each stage one iteration after its MMAs
+// were committed; warps 1-4 prefetch the matching slices of o with cp.async,
+// write them as swizzled bf16 hi/lo tiles into a matching ring and, at the
+// end, read the accumulator out of TMEM.
 // The K dimension is split over the CTAs of a thread-block cluster; their
 // partial tiles are summed through distributed shared memory in a fixed
 // order (deterministic), each CTA writing a slice of the output rows.
@@ -26,7 +28,6 @@ namespace bkv {
 
 constexpr int kTcM = 128;        // output columns (rows of Gt) per CTA
 constexpr int kTcK = 64;         // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kTcStages = 4;
 constexpr int kTcThreads = 160;  // warp 0: TMA + MMA; warps 1-4: o producers + epilogue
 constexpr uint32_t kTcABytes = kTcM * kTcK * 2;
 
@@ -44,10 +45,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
           "r"(smem_u32(dst)),
       "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -110,17 +107,34 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(pred ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// ring depth per batch tile width (shared memory: A 16 KB, B 2*NB*128 B, o staging NB*256 B per stage)
+template <int NB>
+struct TcStages {
+  static constexpr int S = NB <= 16 ? 8 : NB <= 32 ? 6 : 4;
+};
+
 template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     out_proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, OutProjTcParams p) {
-  constexpr int S = kTcStages;
-  constexpr uint32_t kBBytes = NB * kTcK * 2;  // one of hi / lo per stage
+  constexpr int S = TcStages<NB>::S;
+  constexpr uint32_t kBBytes = NB * kTcK * 2;       // one of hi / lo per stage
+  constexpr uint32_t kStageF32 = NB * kTcK * 4;     // fp32 staging of o per stage
+  constexpr int kChunks = NB * 8 / 128;            // 8-float chunks per producer thread per stage
   constexpr uint32_t kCols = NB <= 32 ? 32 : 64;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sA = smem;
   unsigned char* sB = smem + S * kTcABytes;
-  uint64_t* afull = reinterpret_cast<uint64_t*>(sB + S * 2 * kBBytes);
+  unsigned char* sO = sB + S * 2 * kBBytes;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(sO + S * kStageF32);
   uint64_t* bfull = afull + S;
   uint64_t* empty = bfull + S;
   uint64_t* done = empty + S;
@@ -166,7 +180,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_arrive_expect_tx(&afull[i], kTcABytes);
         tma_load_2d(sA + i * kTcABytes, &tmA, (ch0 + i) * kTcK, c0, &afull[i]);
       }
-      for (int i = 0; i < nst && ok; ++i) {
+      for (int i = 0; i < nst; ++i) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)((i / S) & 1);
         if (!mbar_wait_bounded(&afull[s], ph) || !mbar_wait_bounded(&bfull[s], ph)) {
@@ -184,42 +198,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_mma(tmem, ad + step, bl + step, idesc, 1u);
         }
         tc_commit(&empty[s]);
-        if (i + S < nst) {
-          if (!mbar_wait_bounded(&empty[s], ph)) {
+        // refill the stage of the previous iteration (its MMAs have had a whole iteration to finish)
+        const int ip = i - 1;
+        if (ip >= 0 && ip + S < nst) {
+          const int sp = ip % S;
+          if (!mbar_wait_bounded(&empty[sp], (uint32_t)((ip / S) & 1))) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&afull[s], kTcABytes);
-          tma_load_2d(sA + s * kTcABytes, &tmA, (ch0 + i + S) * kTcK, c0, &afull[s]);
+          mbar_arrive_expect_tx(&afull[sp], kTcABytes);
+          tma_load_2d(sA + sp * kTcABytes, &tmA, (ch0 + ip + S) * kTcK, c0, &afull[sp]);
         }
       }
       tc_commit(done);  // arrives when every MMA issued above has completed
     }
     __syncwarp();
   } else {
-    // o producers: 128 threads write the bf16 hi / lo tiles of stage i
+    // o producers: each of the 128 threads owns kChunks 8-float chunks of every
+    // stage; they are prefetched S stages ahead with cp.async into fp32 staging,
+    // then split into bf16 hi / lo and written in the operand's swizzled layout
     const int t = threadIdx.x - 32;
-    for (int i = 0; i < nst && ok; ++i) {
+    auto issue = [&](int i) {
+      unsigned char* stg = sO + (i % S) * kStageF32;
+#pragma unroll
+      for (int m = 0; m < kChunks; ++m) {
+        const int idx = t + 128 * m;
+        const int n = idx >> 3, c = idx & 7;
+        const bool in = b0 + n < p.batch;
+        const float* src = p.o + (in ? (size_t)(b0 + n) * p.K + (size_t)(ch0 + i) * kTcK + c * 8 : 0);
+        cp_async16(stg + n * 256 + c * 32, src, in);
+        cp_async16(stg + n * 256 + c * 32 + 16, src + 4, in);
+      }
+    };
+    for (int i = 0; i < S; ++i) {
+      if (i < nst) issue(i);
+      cp_async_commit();
+    }
+    for (int i = 0; i < nst; ++i) {
       const int s = i % S;
+      cp_async_wait<S - 1>();  // this thread's chunks of stage i have landed
       if (i >= S && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / S) - 1) & 1))) {
         ok = false;
         break;
       }
-      const int kc = ch0 + i;
+      const unsigned char* stg = sO + s * kStageF32;
       unsigned char* hi_t = sB + s * 2 * kBBytes;
       unsigned char* lo_t = hi_t + kBBytes;
-      for (int idx = t; idx < NB * 8; idx += 128) {
-        const int n = idx >> 3, c = idx & 7;
-        float v[8];
-        if (b0 + n < p.batch) {
-          const float4* src = reinterpret_cast<const float4*>(p.o + (size_t)(b0 + n) * p.K + kc * kTcK + c * 8);
-          const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
-          v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-          v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
-        } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = 0.f;
-        }
+      for (int m = 0; m < kChunks; ++m) {
+        const int idx = t + 128 * m;
+        const int n = idx >> 3, c = idx & 7;
+        const float4 x0 = *reinterpret_cast<const float4*>(stg + n * 256 + c * 32);
+        const float4 x1 = *reinterpret_cast<const float4*>(stg + n * 256 + c * 32 + 16);
+        const float v[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -235,7 +266,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(&bfull[s]);
+      if (i + S < nst) issue(i + S);  // the staging slot of stage i is free again
+      cp_async_commit();
     }
+    cp_async_wait<0>();
   }
 
   // accumulator complete
@@ -340,8 +374,10 @@ bool out_proj_tc_supported(int K, int hidden, int batch) {
   return K % kTcK == 0 && hidden % kTcM == 0 && batch >= 1 && encode_fn() != nullptr;
 }
 
-static size_t tc_smem_bytes(int NB) {
-  return 1024 + (size_t)kTcStages * kTcABytes + (size_t)kTcStages * 2 * NB * kTcK * 2 + (3 * kTcStages + 1) * 8 + 16;
+template <int NB>
+static size_t tc_smem_bytes() {
+  constexpr int S = TcStages<NB>::S;
+  return 1024 + (size_t)S * kTcABytes + (size_t)S * 2 * NB * kTcK * 2 + (size_t)S * NB * kTcK * 4 + (3 * S + 1) * 8 + 16;
 }
 
 template <int NB>
@@ -353,7 +389,7 @@ static cudaError_t launch_tc_nb(const CUtensorMap& map, OutProjTcParams p, int n
   while (ks * 2 <= 8 && ks * 2 <= KC && (long long)mtiles * bchunks * ks * 2 <= num_sms) ks *= 2;
   p.ksplit = ks;
   p.chunks_per_cta = (KC + ks - 1) / ks;
-  const size_t smem = tc_smem_bytes(NB);
+  const size_t smem = tc_smem_bytes<NB>();
   cudaError_t e = ensure_smem((const void*)out_proj_tc_kernel<NB>, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

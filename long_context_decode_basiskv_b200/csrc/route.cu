@@ -12,10 +12,13 @@
 // transpose-reduction leaves one (page, head) score per lane.  The summary of
 // a page is read once for the whole GQA group.  HBM-bound.
 //
-// Kernel 2 (select): one CTA per (sequence, query head) runs an exact radix
-// select (4 passes of 8 bits) on order-preserving integer keys of the fp32
-// scores, then resolves ties at the threshold by ascending page index and
-// compacts the kept pages in ascending order with two block scans.
+// Kernel 2 (select): one CTA per (sequence, query head) finds T, the exact
+// k-th largest score: a 256-bucket histogram over the linear score range (a
+// monotone map, so whole buckets above the boundary bucket are kept) narrows
+// the search to the boundary bucket, refined up to three times, whose few
+// scores are ranked exactly.  Pages scoring above T are kept, ties at T go to
+// the lowest page indices, and a block scan compacts the kept pages (plus the
+// sink and recent pages) in ascending order.
 #include "kernels.cuh"
 
 namespace bkv {
@@ -55,7 +58,8 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
       for (int u = 0; u < DPL; ++u) qf[hi][u] = Elem<T>::to_f(qb[hi * D + lane * DPL + u]);
 
     int my_phys = -1;
-    if (lane < kPagesPerWarp && p0 + lane < n) {
+    const int pl = p0 + lane;
+    if (lane < kPagesPerWarp && pl < n && (p.all_pages || (pl != 0 && pl != n - 1))) {
       my_phys = p.block_table[(size_t)b * p.max_pages + p0 + lane];
       if (my_phys < 0 || my_phys >= p.num_phys) {
         set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
       const int idx = lane / kDup;
       const int i = idx / G, hi = idx % G;
       const int ph = __shfl_sync(kFull, my_phys, i);
-      if ((lane % kDup) == 0 && p0 + i < n)
+      if ((lane % kDup) == 0 && p0 + i < n && ph != -1)
         out[(size_t)hi * p.max_pages + i] = (ph == -2) ? -INFINITY : part[0];
     } else {
 #pragma unroll
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
         const int idx = 2 * lane + j;
         const int i = idx / G, hi = idx % G;
         const int ph = __shfl_sync(kFull, my_phys, i);
-        if (p0 + i < n) out[(size_t)hi * p.max_pages + i] = (ph == -2) ? -INFINITY : part[j];
+        if (p0 + i < n && ph != -1) out[(size_t)hi * p.max_pages + i] = (ph == -2) ? -INFINITY : part[j];
       }
     }
   }
@@ -115,26 +119,60 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
 // ---------------------------------------------------------------------------
 // selection
 // ---------------------------------------------------------------------------
-
-
 constexpr int kSelectThreads = 256;
+constexpr int kCandCap = 512;  // boundary candidates ranked exactly in shared memory
+constexpr int kLevels = 3;     // histogram refinements of the boundary bucket
 
-// order-preserving map fp32 -> uint32 (larger score -> larger key); -0 == +0
-__device__ __forceinline__ uint32_t order_key(float x) {
-  if (x == 0.f) x = 0.f;
-  const uint32_t u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+// Monotone map of a score to one of 256 linear buckets over [lo, lo + 255.99/inv]:
+// s1 <= s2 implies bucket(s1) <= bucket(s2) (fp subtraction, scaling and the
+// clamps are all monotone), so every score in a higher bucket is larger.
+__device__ __forceinline__ int lin_bucket(float s, float lo, float inv) {
+  const float x = fminf(fmaxf((s - lo) * inv, 0.f), 255.f);  // fmaxf maps NaN to 0
+  return (int)x;
 }
 
+__device__ __forceinline__ void block_minmax(float& mn, float& mx, float* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  mn = -warp_max(-mn);
+  mx = warp_max(mx);
+  if (lane == 0) {
+    red[w] = mn;
+    red[32 + w] = mx;
+  }
+  __syncthreads();
+  float a = (lane < nw) ? red[lane] : INFINITY, c = (lane < nw) ? red[32 + lane] : -INFINITY;
+  mn = -warp_max(-a);
+  mx = warp_max(c);
+  __syncthreads();
+}
+
+__device__ __forceinline__ int block_sum(int v, int* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  int t = (lane < nw) ? red[lane] : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
+  __syncthreads();
+  return t;
+}
+
+// One CTA per (sequence, query head).  Finds T, the k-th largest score of
+// pages 1..n-2, and how many pages scoring exactly T are kept (the lowest
+// indices), then writes the kept pages plus 0 and n-1 in ascending order.
 __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(SelectParams p) {
-  extern __shared__ __align__(16) uint32_t keys[];  // [max_pages]
+  extern __shared__ __align__(16) float ssc[];  // [max_pages] scores of this head
   __shared__ int hist[256];
   __shared__ int warp_tot[32];
-  __shared__ uint32_t s_digit;
-  __shared__ int s_above;
+  __shared__ float redf[64];
+  __shared__ float cand[kCandCap];
+  __shared__ int s_ncand, s_D, s_above, s_rem;
+  __shared__ float s_T;
 
   const int h = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int L = p.seq_len[b];
   const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
   const int kk = p.top_k;
@@ -147,97 +185,156 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(SelectPara
     if (tid == 0) p.sel_cnt[row] = n;
     return;
   }
+  const int ncand = n - 2;  // pages 1 .. n-2 compete
 
-  const int ncand = n - 2;  // pages 1 .. n-2
-  for (int i = tid; i < ncand; i += blockDim.x) keys[1 + i] = order_key(sc[1 + i]);
-  __syncthreads();
-
-  uint32_t prefix = 0, pmask = 0;
-  int rem = kk;  // how many of the matching keys are still to be taken
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  float mn = INFINITY, mx = -INFINITY;
+  for (int i = tid; i < ncand; i += blockDim.x) {
+    float v = sc[1 + i];
+    if (v == 0.f) v = 0.f;  // -0 == +0
+    ssc[1 + i] = v;
+    if (isfinite(v)) {
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+    }
+  }
+  block_minmax(mn, mx, redf);  // also orders the stores to ssc before the reads below
+  float lo = (mn <= mx) ? mn : 0.f, hi = (mn <= mx) ? mx : 0.f;
+  int rem = kk;   // how many of the still-undecided candidates are kept
+  int D = 0;      // boundary bucket of the last level
+  float inv = 0.f;
+  int level = 0;
+  for (;; ++level) {
     for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int base = 0; base < ncand; base += blockDim.x) {
-      const int i = base + tid;
-      uint32_t digit = 0xffffffffu;
-      if (i < ncand) {
-        const uint32_t key = keys[1 + i];
-        if ((key & pmask) == prefix) digit = (key >> shift) & 0xffu;
-      }
-      const unsigned same = __match_any_sync(kFull, digit);
-      if (digit != 0xffffffffu && lane == __ffs(same) - 1) atomicAdd(&hist[digit], __popc(same));
+    inv = (hi > lo) ? 255.99f / (hi - lo) : 0.f;
+    if (!isfinite(inv)) inv = 0.f;
+    for (int i = tid; i < ncand; i += blockDim.x) {
+      const float v = ssc[1 + i];
+      if (level == 0 || (v >= lo && v <= hi)) atomicAdd(&hist[lin_bucket(v, lo, inv)], 1);
     }
     __syncthreads();
     if (tid < 32) {
-      // lane owns digits 8*lane .. 8*lane+7; count of matching keys above each digit
-      int loc[8];
-      int sum = 0;
+      int loc[8], sum = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         loc[j] = hist[8 * tid + j];
         sum += loc[j];
       }
-      int above = 0;  // sum over lanes with higher digits
       int x = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_down_sync(kFull, x, o);
         if (tid + o < 32) x += y;
       }
-      above = x - sum;  // inclusive suffix minus own
+      int above = x - sum;
 #pragma unroll
       for (int j = 7; j >= 0; --j) {
         if (above < rem && rem <= above + loc[j]) {
-          s_digit = (uint32_t)(8 * tid + j);
+          s_D = 8 * tid + j;
           s_above = above;
         }
         above += loc[j];
       }
     }
     __syncthreads();
-    prefix |= s_digit << shift;
-    pmask |= 0xffu << shift;
+    D = s_D;
     rem -= s_above;
-    __syncthreads();
+    const int c = hist[D];
+    if (c <= kCandCap || inv == 0.f || level + 1 >= kLevels) break;
+    // refine: the scores of bucket D form an interval; histogram it again
+    float bmn = INFINITY, bmx = -INFINITY;
+    for (int i = tid; i < ncand; i += blockDim.x) {
+      const float v = ssc[1 + i];
+      if ((level == 0 || (v >= lo && v <= hi)) && lin_bucket(v, lo, inv) == D) {
+        bmn = fminf(bmn, v);
+        bmx = fmaxf(bmx, v);
+      }
+    }
+    block_minmax(bmn, bmx, redf);
+    if (!(isfinite(bmn) && isfinite(bmx))) break;  // an infinite score in the bucket: rank it exactly
+    lo = bmn;
+    hi = bmx;
   }
-  const uint32_t thr = prefix;  // key of the k-th largest candidate
-  // rem = how many candidates equal to thr are kept (lowest page index first)
 
-  // pass A: rank of each equal-to-threshold candidate in page order
+  // the boundary candidates: the level's active scores in bucket D
+  auto in_boundary = [&](float v) {
+    return (level == 0 || (v >= lo && v <= hi)) && lin_bucket(v, lo, inv) == D;
+  };
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
+  const int c = hist[D];
+  if (c <= kCandCap) {
+    for (int i = tid; i < ncand; i += blockDim.x) {
+      const float v = ssc[1 + i];
+      if (in_boundary(v)) cand[atomicAdd(&s_ncand, 1)] = v;
+    }
+    __syncthreads();
+    for (int i = tid; i < c; i += blockDim.x) {
+      const float v = cand[i];
+      int gt = 0, eq = 0;
+      for (int j = 0; j < c; ++j) {
+        gt += cand[j] > v;
+        eq += cand[j] == v;
+      }
+      if (gt < rem && rem <= gt + eq) {
+        s_T = v;
+        s_rem = rem - gt;
+      }
+    }
+  } else {
+    // many equal (or infinite) scores in one bucket: rank against every boundary score
+    for (int i = tid; i < ncand; i += blockDim.x) {
+      const float v = ssc[1 + i];
+      if (!in_boundary(v)) continue;
+      int gt = 0, eq = 0;
+      for (int j = 0; j < ncand; ++j) {
+        const float w = ssc[1 + j];
+        if (in_boundary(w)) {
+          gt += w > v;
+          eq += w == v;
+        }
+      }
+      if (gt < rem && rem <= gt + eq) {
+        s_T = v;
+        s_rem = rem - gt;
+      }
+    }
+  }
+  __syncthreads();
+  const float T = s_T;
+  const int keep_eq = s_rem;  // candidates scoring exactly T that are kept
+
+  // ties at T: the lowest page indices win
   const int per = (n + kSelectThreads - 1) / kSelectThreads;
-  const int lo = tid * per, hi = min(n, lo + per);
+  const int plo = tid * per, phi = min(n, plo + per);
   int eq_local = 0;
-  for (int pg = lo; pg < hi; ++pg)
-    if (pg >= 1 && pg <= n - 2 && keys[pg] == thr) ++eq_local;
-  int tot;
-  int eq_rank = block_exclusive_scan(eq_local, warp_tot, tot);
-  // pass B: keep flags and their count
+  for (int pg = plo; pg < phi; ++pg)
+    if (pg >= 1 && pg <= n - 2 && ssc[pg] == T) ++eq_local;
+  const int eq_total = block_sum(eq_local, warp_tot);
+  int eq_rank = 0, tot = 0;
+  if (eq_total > keep_eq) eq_rank = block_exclusive_scan(eq_local, warp_tot, tot);
   int take_local = 0;
   {
     int er = eq_rank;
-    for (int pg = lo; pg < hi; ++pg) {
-      bool take;
-      if (pg == 0 || pg == n - 1) {
-        take = true;
-      } else {
-        const uint32_t key = keys[pg];
-        take = key > thr || (key == thr && er < rem);
-        if (key == thr) ++er;
+    for (int pg = plo; pg < phi; ++pg) {
+      bool take = (pg == 0 || pg == n - 1);
+      if (!take) {
+        const float v = ssc[pg];
+        take = v > T || (v == T && er < keep_eq);
+        if (v == T) ++er;
       }
-      take_local += take ? 1 : 0;
+      take_local += take;
     }
   }
   int pos = block_exclusive_scan(take_local, warp_tot, tot);
   {
     int er = eq_rank;
-    for (int pg = lo; pg < hi; ++pg) {
-      bool take;
-      if (pg == 0 || pg == n - 1) {
-        take = true;
-      } else {
-        const uint32_t key = keys[pg];
-        take = key > thr || (key == thr && er < rem);
-        if (key == thr) ++er;
+    for (int pg = plo; pg < phi; ++pg) {
+      bool take = (pg == 0 || pg == n - 1);
+      if (!take) {
+        const float v = ssc[pg];
+        take = v > T || (v == T && er < keep_eq);
+        if (v == T) ++er;
       }
       if (take) out[pos++] = pg;
     }
@@ -278,7 +375,7 @@ cudaError_t launch_route(const ScoreParams& sp, const SelectParams& selp, int d,
                    : launch_score_g<float, 64>(sp, G, (int)blocks, st);
   }
   if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)sp.max_pages * sizeof(uint32_t);
+  const size_t smem = (size_t)sp.max_pages * sizeof(float);
   e = ensure_smem((const void*)route_select_kernel, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(sp.Hq, sp.batch);

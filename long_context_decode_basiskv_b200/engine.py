@@ -76,10 +76,27 @@ class DecodeEngine:
     def out_proj(self, stream=None):
         bk.out_proj(self.cfg, self.factors, self.o_lat, self.y, self.ws, stream)
 
+    def append_route(self, stream=None):
+        """Append (on a forked stream) concurrently with route, then join.
+
+        Without a scores output, route reads nothing the step's append writes
+        (only the recent page changes, and it is kept whatever it scores).
+        """
+        main = torch.cuda.current_stream(self.device) if stream is None else stream
+        if not hasattr(self, "_aux"):
+            self._aux = torch.cuda.Stream(device=self.device)
+            self._fork = torch.cuda.Event()
+            self._join = torch.cuda.Event()
+        self._fork.record(main)
+        self._aux.wait_event(self._fork)
+        self.append(self._aux)
+        self._join.record(self._aux)
+        self.route(stream=main)
+        main.wait_event(self._join)
+
     def step(self, stream=None):
-        """One decode step: append -> route -> decode_attn -> out_proj (one stream)."""
-        self.append(stream)
-        self.route(stream=stream)
+        """One decode step: (append || route) -> decode_attn -> out_proj."""
+        self.append_route(stream)
         self.decode_attn(stream)
         self.out_proj(stream)
         return self.y
