@@ -119,9 +119,14 @@ typedef struct {
 /*
  * Factors (device, dtype).  A [Hkv][d][r] (Value -> latent), P [Hkv][r][d]
  * (latent -> predicted key), E [Hkv][d][s] (key residual basis),
- * Gt [hidden][Hq][r]: the fused out-projection factor G_h = B_g(h) W_O,h,
- * stored transposed (row c holds output column c for every head and latent
- * dimension); basiskv_fuse_out_factor writes it.
+ * Gt: the fused out-projection factor G_h = B_g(h) W_O,h, hidden * Hq * r
+ * elements written by basiskv_fuse_out_factor.  Element (c, k), output column
+ * c and k = h * r + i, K = Hq * r, sits at
+ *   - bf16 with K % 64 == 0 and hidden % 128 == 0 (the tensor-core layout):
+ *     ((c/128 * K/64 + k/64) * 128 + c%128) * 64 + ((k%64/8) ^ (c%8)) * 8 + k%8,
+ *     i.e. 128 x 64 tiles, each a contiguous 16 KB block whose 128-byte rows
+ *     hold their 16-byte chunks in XOR-swizzled order;
+ *   - every other shape: c * K + k (row-major [hidden][Hq][r]).
  */
 typedef struct {
   const void* A;
@@ -216,10 +221,11 @@ BASISKV_API basiskv_status basiskv_out_proj(const basiskv_config* cfg, const bas
                                 size_t workspace_bytes, void* stream);
 
 /*
- * Weight preparation for step 5 (not per step).  Gt[c][h][i] =
+ * Weight preparation for step 5 (not per step).  Gt(c, h r + i) =
  * sum_j Bf[g(h)][i][j] W_O[h d + j][c], accumulated in fp64 and rounded once to
- * dtype.  Bf (device, dtype) [Hkv][r][d]; W_O (device, dtype) [Hq d][hidden];
- * Gt (device, dtype) [hidden][Hq][r].
+ * dtype, stored in the layout described with basiskv_factors.  Bf (device,
+ * dtype) [Hkv][r][d]; W_O (device, dtype) [Hq d][hidden]; Gt (device, dtype)
+ * hidden * Hq * r elements.
  */
 BASISKV_API basiskv_status basiskv_fuse_out_factor(const basiskv_config* cfg, const void* Bf,
                                        const void* W_O, void* Gt, void* stream);

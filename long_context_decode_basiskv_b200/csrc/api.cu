@@ -63,7 +63,8 @@ static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 // routing scores first, then the decode scratch of decode_plan()
 static Workspace layout(const basiskv_config* c, int batch, int max_pages) {
   Workspace w{};
-  w.plan = decode_plan(c->num_q_heads, c->num_kv_heads, c->page_size, c->rank_v, c->top_k, batch, max_pages);
+  w.plan = decode_plan(c->num_q_heads, c->num_kv_heads, c->page_size, c->rank_v, c->top_k, batch, max_pages,
+                       c->dtype == BASISKV_BF16, c->head_dim);
   w.scores = 0;
   w.decode = up256((size_t)batch * c->num_q_heads * max_pages * 4);
   w.total = w.decode + w.plan.bytes;
@@ -167,7 +168,7 @@ basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors
   (void)ws;
   (void)ws_bytes;
   const int K = cfg->num_q_heads * cfg->rank_v;
-  if (cfg->dtype == BASISKV_BF16 && out_proj_tc_supported(K, cfg->hidden, batch))
+  if (cfg->dtype == BASISKV_BF16 && gt_blocked(K, cfg->hidden))
     return cuda_status(launch_out_proj_tc(o_lat, f->Gt, y, nullptr, batch, K, cfg->hidden, num_sms(),
                                           (cudaStream_t)stream));
   OutProjParams p{o_lat, f->Gt, y, batch, K, cfg->hidden};
@@ -179,7 +180,9 @@ basiskv_status basiskv_fuse_out_factor(const basiskv_config* cfg, const void* Bf
   basiskv_status s = check_config(cfg);
   if (s != BASISKV_OK) return s;
   if (!Bf || !W_O || !Gt) return BASISKV_ERR_INVALID_ARG;
-  FuseParams p{Bf, W_O, Gt, cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->hidden};
+  const bool blocked = cfg->dtype == BASISKV_BF16 && gt_blocked(cfg->num_q_heads * cfg->rank_v, cfg->hidden);
+  FuseParams p{Bf, W_O, Gt, cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->hidden,
+               blocked ? 1 : 0};
   return cuda_status(launch_fuse(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
 }
 

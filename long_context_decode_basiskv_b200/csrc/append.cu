@@ -69,6 +69,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendParams p) 
   T* cdst = static_cast<T*>(p.c_lat) + blk * P * r;
   T* rdst = static_cast<T*>(p.r_res) + blk * P * s;
 
+  // bf16 K and C rows are stored swizzled for the tensor-core attention path
+  const bool swz_on = kc_swizzled(sizeof(T) == 2, d, r);
+  const int mk = swz_on ? swz_mask(d) : 0, mc = swz_on ? swz_mask(r) : 0;
   const int t_lo = max(first_new, page * P);
   const int t_hi = min(L, (page + 1) * P);
   const T* kin = static_cast<const T*>(p.k_new);
@@ -83,7 +86,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendParams p) 
       const T kv = kin[row * d + x];
       sk[t * d + x] = Elem<T>::to_f(kv);
       sv[t * d + x] = Elem<T>::to_f(vin[row * d + x]);
-      kdst[(size_t)(c0 + t - page * P) * d + x] = kv;  // raw key stored as given
+      const int slot = c0 + t - page * P;
+      kdst[(size_t)slot * d + swz(x, slot, mk)] = kv;  // raw key stored as given
     }
     __syncthreads();
     // C = v A
@@ -92,7 +96,8 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendParams p) 
       double acc = 0.0;
       for (int x = 0; x < d; ++x) acc = fma((double)sv[t * d + x], Elem<T>::to_d(sA[x * r + j]), acc);
       sC[t * r + j] = acc;
-      cdst[(size_t)(c0 + t - page * P) * r + j] = Elem<T>::from_d(acc);
+      const int slot = c0 + t - page * P;
+      cdst[(size_t)slot * r + swz(j, slot, mc)] = Elem<T>::from_d(acc);
     }
     __syncthreads();
     // U = k - C P   (C unrounded)
@@ -118,7 +123,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(AppendParams p) 
   for (int j = tid; j < r + s; j += blockDim.x) {
     double acc = 0.0;
     if (j < r) {
-      for (int t = 0; t < m; ++t) acc += Elem<T>::to_d(cdst[(size_t)t * r + j]);
+      for (int t = 0; t < m; ++t) acc += Elem<T>::to_d(cdst[(size_t)t * r + swz(j, t, mc)]);
     } else {
       for (int t = 0; t < m; ++t) acc += Elem<T>::to_d(rdst[(size_t)t * s + (j - r)]);
     }

@@ -35,6 +35,22 @@ template <> struct Elem<__nv_bfloat16> {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Row swizzle of bf16 K and C pages for the tensor-core attention path: the
+// 16-byte chunk c of page row j is stored at chunk c ^ (j & mask), which keeps
+// 8 consecutive rows of one chunk column in 8 different bank groups.  mask is
+// the largest of 7, 3, 1 that keeps every chunk inside its row.
+__host__ __device__ __forceinline__ int swz_mask(int row_elems) {
+  const int chunks = row_elems / 8;
+  return (chunks % 8 == 0) ? 7 : (chunks % 4 == 0) ? 3 : (chunks % 2 == 0) ? 1 : 0;
+}
+__host__ __device__ __forceinline__ int swz(int x, int row, int mask) {
+  return ((((x >> 3) ^ (row & mask)) << 3) | (x & 7));
+}
+// K and C pages are swizzled exactly when the tensor-core attention path runs
+__host__ __device__ __forceinline__ bool kc_swizzled(bool bf16, int d, int r) {
+  return bf16 && d % 16 == 0 && r % 16 == 0;
+}
+
 __device__ __forceinline__ void set_err(int32_t* flag, int32_t bits) {
   if (flag) atomicOr(flag, bits);
 }

@@ -39,8 +39,9 @@ constexpr int kTargetCtas = 888;    // one wave of attn CTAs on a B200 (148 SMs 
 // ---------------------------------------------------------------------------
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages) {
+DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d) {
   DecodePlan pl{};
+  const int target = kc_swizzled(bf16, d, r) ? 444 : kTargetCtas;  // CTAs per wave of the kernel that runs
   const int G = Hq / Hkv;
   long long um = (long long)G * (top_k + 2);
   if (um > max_pages) um = max_pages;
@@ -48,7 +49,7 @@ DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, i
   pl.tpp = page / kTile;
   const long long groups = (long long)batch * Hkv;
   const long long tiles = (long long)pl.umax * pl.tpp;
-  long long eps = (tiles * groups + kTargetCtas - 1) / kTargetCtas;  // tiles per split, then pages
+  long long eps = (tiles * groups + target - 1) / target;  // tiles per split, then pages
   eps = (eps + pl.tpp - 1) / pl.tpp;
   if (eps < 1) eps = 1;
   pl.eps = (int)eps;
@@ -152,6 +153,36 @@ __device__ __forceinline__ void load_pair(const T* row, int dim, float& a, float
     const float2 w = *reinterpret_cast<const float2*>(row + dim);
     a = w.x;
     b = w.y;
+  }
+}
+
+// The last CTA of a (sequence, KV head) group merges the group's split
+// results: for each of its G heads, log-sum-exp over the splits.  Heads are
+// spread over `nw` warps starting at warp index `wi`.
+__device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, int g, int G, int r,
+                                                   int nsplit_active, int wi, int nw, int lane) {
+  for (int hi = wi; hi < G; hi += nw) {
+    const int h = g * G + hi;
+    const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * (r + 2);
+    float M = -INFINITY;
+    for (int s = lane; s < nsplit_active; s += 32) M = fmaxf(M, __ldcg(base + (size_t)s * (r + 2)));
+    M = warp_max(M);
+    float Ls = 0.f;
+    for (int s = lane; s < nsplit_active; s += 32) {
+      const float ms = __ldcg(base + (size_t)s * (r + 2));
+      if (ms != -INFINITY) Ls += __ldcg(base + (size_t)s * (r + 2) + 1) * exp2f(ms - M);
+    }
+    Ls = warp_sum(Ls);
+    for (int dim = lane; dim < r; dim += 32) {
+      float a = 0.f;
+      if (M != -INFINITY)
+        for (int s = 0; s < nsplit_active; ++s) {
+          const float* ps = base + (size_t)s * (r + 2);
+          const float ms = __ldcg(ps);
+          if (ms != -INFINITY) a += __ldcg(ps + 2 + dim) * exp2f(ms - M);
+        }
+      p.o_lat[((size_t)b * p.Hq + h) * r + dim] = (Ls > 0.f) ? a / Ls : 0.f;
+    }
   }
 }
 
@@ -343,28 +374,295 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   __syncthreads();
   if (!s_last || warp == 0) return;
   __threadfence();
-  const int hi = warp - 1;
-  const int h = g * G + hi;
-  const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * (r + 2);
-  float M = -INFINITY;
-  for (int s = lane; s < nsplit_active; s += 32) M = fmaxf(M, __ldcg(base + (size_t)s * (r + 2)));
-  M = warp_max(M);
-  float Ls = 0.f;
-  for (int s = lane; s < nsplit_active; s += 32) {
-    const float ms = __ldcg(base + (size_t)s * (r + 2));
-    if (ms != -INFINITY) Ls += __ldcg(base + (size_t)s * (r + 2) + 1) * exp2f(ms - M);
+  merge_group_splits(p, b, g, G, r, nsplit_active, warp - 1, G, lane);
+}
+
+// ---------------------------------------------------------------------------
+// bf16 path: one consumer warp per tile, all G heads of the group at once on
+// the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate)
+//   S^T[16 x 16] = Q[16 (heads, padded) x d] . K_tile^T[d x 16 tokens]
+//   O[16 x r]   += P[16 x 16 tokens] . C_tile[16 tokens x r]
+// P reuses the S^T accumulator registers as the A operand (the m16n8k16 C and
+// A fragments line up), rounded to bf16.  K and C rows are XOR-swizzled in the
+// page (see swz()), so ldmatrix reads 8 rows without bank conflicts.
+// ---------------------------------------------------------------------------
+constexpr int kMmaWarps = 4;       // warps per CTA; each streams and consumes its own tiles
+constexpr int kMmaWarpStages = 3;  // ring slots per warp
+constexpr int kMmaTargetCtas = 444;  // one wave at 3 CTAs per SM
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int D, int G, int NT>
+__global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams p) {
+  constexpr int KS = D / 16;
+  constexpr int SW = kMmaWarpStages;
+  constexpr int R = NT * 8;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_last;
+  __shared__ uint32_t meta_all[kMmaWarps][kMmaWarpStages];  // head mask | valid << 8 of each slot's tile
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t* meta = meta_all[w];
+  const size_t bg = (size_t)b * p.Hkv + g;
+  const int U = p.ucnt[bg];
+  const int e0 = split * p.eps;
+  const int nsplit_active = (U + p.eps - 1) / p.eps;
+  if (e0 >= U) {
+    if (split == 0 && U == 0)
+      for (int i = threadIdx.x; i < G * R; i += blockDim.x)
+        p.o_lat[((size_t)b * p.Hq + (size_t)g * G) * R + i] = 0.f;
+    return;
   }
-  Ls = warp_sum(Ls);
-  for (int dim = lane; dim < r; dim += 32) {
-    float a = 0.f;
-    if (M != -INFINITY)
-      for (int s = 0; s < nsplit_active; ++s) {
-        const float* ps = base + (size_t)s * (r + 2);
-        const float ms = __ldcg(ps);
-        if (ms != -INFINITY) a += __ldcg(ps + 2 + dim) * exp2f(ms - M);
+  const int nent = min(U, e0 + p.eps) - e0;
+  const int ntiles = nent * p.tpp;
+
+  constexpr uint32_t k_bytes = kTile * D * 2;
+  constexpr uint32_t c_bytes = kTile * R * 2;
+  constexpr uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
+  unsigned char* ring = smem + (size_t)w * SW * stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kMmaWarps * SW * stage_bytes) + w * SW;
+  if (lane == 0) {
+    for (int s = 0; s < SW; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const int L = p.seq_len[b];
+  const int n = min((L + p.page - 1) / p.page, p.max_pages);
+  const int last_valid = L - (n - 1) * p.page;
+  const int32_t* uni = p.uni + bg * p.umax;
+  const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k_raw);
+  const __nv_bfloat16* cbase = static_cast<const __nv_bfloat16*>(p.c_lat);
+
+  // this warp's tiles: t = w + kMmaWarps * i; lane j of a batch of 32 holds tile i = base + j
+  const int my_tiles = (ntiles > w) ? (ntiles - w + kMmaWarps - 1) / kMmaWarps : 0;
+  int d_phys = -1, d_valid = 0;
+  uint32_t d_mask = 0;
+  auto load_desc = [&](int base) {  // descriptors of tiles base .. base+31 of this warp
+    d_phys = -1;
+    d_valid = 0;
+    d_mask = 0;
+    const int i = base + lane;
+    if (i < my_tiles) {
+      const int t = w + kMmaWarps * i;
+      const int e = t / p.tpp, sub = t - e * p.tpp;
+      const uint32_t ent = (uint32_t)uni[e0 + e];
+      const int pg = (int)(ent & 0xffffffu);
+      d_mask = ent >> 24;
+      if (pg < n) {
+        const int ph = p.block_table[(size_t)b * p.max_pages + pg];
+        if (ph >= 0 && ph < p.num_phys) {
+          d_phys = ph * p.tpp + sub;  // tile index of the head-g page block, in 16-row units
+          d_valid = min(kTile, max(0, ((pg == n - 1) ? last_valid : p.page) - sub * kTile));
+        } else {
+          set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
+        }
       }
-    p.o_lat[((size_t)b * p.Hq + h) * r + dim] = (Ls > 0.f) ? a / Ls : 0.f;
+    }
+  };
+  // issue tile i of this warp into slot i % SW (lane 0); all lanes take part in the shuffles
+  auto issue = [&](int i) {
+    const int j = i & 31;
+    const int ph = __shfl_sync(kFull, d_phys, j);
+    const int valid = __shfl_sync(kFull, d_valid, j);
+    const uint32_t mask = __shfl_sync(kFull, d_mask, j);
+    if (lane == 0) {
+      meta[i % SW] = mask | ((uint32_t)valid << 8);
+      uint64_t* bar = &full[i % SW];
+      unsigned char* st = ring + (size_t)(i % SW) * stage_bytes;
+      fence_proxy_async_smem();
+      if (valid > 0) {
+        const int pidx = ph / p.tpp, sub = ph - pidx * p.tpp;
+        const size_t row0 = ((size_t)pidx * p.Hkv + g) * p.page + (size_t)sub * kTile;
+        mbar_arrive_expect_tx(bar, k_bytes + c_bytes);
+        bulk_g2s(st, kbase + row0 * D, k_bytes, bar);
+        bulk_g2s(st + k_bytes, cbase + row0 * R, c_bytes, bar);
+      } else {
+        mbar_arrive_expect_tx(bar, 0);
+      }
+    }
+  };
+
+  const int gr = lane >> 2, tq = lane & 3;  // fragment row (head) and column pair
+  const bool head_ok = gr < G;
+  uint32_t qa[KS][2];
+  {
+    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G + gr) * D;
+#pragma unroll
+    for (int s2 = 0; s2 < KS; ++s2) {
+      qa[s2][0] = head_ok ? *reinterpret_cast<const uint32_t*>(qr + 16 * s2 + 2 * tq) : 0u;
+      qa[s2][1] = head_ok ? *reinterpret_cast<const uint32_t*>(qr + 16 * s2 + 2 * tq + 8) : 0u;
+    }
   }
+  float m_run = -INFINITY, l_run = 0.f;
+  float oacc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+  constexpr int mk = 7;  // K rows have 8 or 16 chunks
+  const int mc = swz_mask(R);
+  const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix mi takes its row rr from this lane
+  bool ok = true;
+
+  if (my_tiles > 0) load_desc(0);
+  for (int i = 0; i < min(SW, my_tiles); ++i) issue(i);
+  for (int i = 0; i < my_tiles; ++i) {
+    const int s = i % SW;
+    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / SW) & 1))) {
+      ok = false;
+      break;
+    }
+    const uint32_t mt = meta[s];
+    const int valid = (int)(mt >> 8);
+    if (valid > 0) {
+      unsigned char* st = ring + (size_t)s * stage_bytes;
+      const uint32_t kaddr = smem_u32(st);
+      const uint32_t caddr = smem_u32(st + k_bytes);
+      if (valid < kTile) {
+        // rows past the valid tokens hold stale bits: zero them (0 * NaN would poison O)
+        for (int x = lane; x < (kTile - valid) * R / 8; x += 32)
+          reinterpret_cast<uint4*>(st + k_bytes)[valid * R / 8 + x] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+      }
+      // S^T = Q K^T, k-steps split over two accumulator chains
+      float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int tok = (mi >> 1) * 8 + rr;
+        const uint32_t rowaddr = kaddr + (uint32_t)(tok * D * 2);
+#pragma unroll
+        for (int s2 = 0; s2 < KS; ++s2) {
+          const int chunk = 2 * s2 + (mi & 1);
+          uint32_t kb[4];
+          ldsm4(kb, rowaddr + (uint32_t)((chunk ^ (tok & mk)) << 4));
+          if (s2 & 1) {
+            mma16816(sb[0], qa[s2][0], qa[s2][1], kb[0], kb[1]);
+            mma16816(sb[1], qa[s2][0], qa[s2][1], kb[2], kb[3]);
+          } else {
+            mma16816(sa[0], qa[s2][0], qa[s2][1], kb[0], kb[1]);
+            mma16816(sa[1], qa[s2][0], qa[s2][1], kb[2], kb[3]);
+          }
+        }
+      }
+      // online softmax on row gr (this lane holds tokens 2tq, 2tq+1, 8+2tq, 9+2tq)
+      const bool row_on = head_ok && ((mt >> gr) & 1u);
+      float sv[4];
+      sv[0] = (row_on && 2 * tq < valid) ? (sa[0][0] + sb[0][0]) * p.qscale : -INFINITY;
+      sv[1] = (row_on && 2 * tq + 1 < valid) ? (sa[0][1] + sb[0][1]) * p.qscale : -INFINITY;
+      sv[2] = (row_on && 8 + 2 * tq < valid) ? (sa[1][0] + sb[1][0]) * p.qscale : -INFINITY;
+      sv[3] = (row_on && 9 + 2 * tq < valid) ? (sa[1][1] + sb[1][1]) * p.qscale : -INFINITY;
+      float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+      const float m_new = fmaxf(m_run, mx);
+      float pr[4], corr = 1.f;
+      if (m_new == -INFINITY) {
+        pr[0] = pr[1] = pr[2] = pr[3] = 0.f;
+      } else {
+        corr = exp2f(m_run - m_new);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) pr[x] = exp2f(sv[x] - m_new);
+      }
+      l_run = l_run * corr + (pr[0] + pr[1] + pr[2] + pr[3]);
+      m_run = m_new;
+#pragma unroll
+      for (int jj = 0; jj < NT; ++jj) {
+        oacc[jj][0] *= corr;
+        oacc[jj][1] *= corr;
+      }
+      // O += P C
+      const uint32_t pa0 = pack_bf16(pr[0], pr[1]), pa2 = pack_bf16(pr[2], pr[3]);
+      {
+        const int tok = (mi & 1) * 8 + rr;
+        const uint32_t rowaddr = caddr + (uint32_t)(tok * R * 2);
+#pragma unroll
+        for (int jj = 0; jj < NT / 2; ++jj) {
+          const int chunk = 2 * jj + (mi >> 1);
+          uint32_t cb4[4];
+          ldsm4t(cb4, rowaddr + (uint32_t)((chunk ^ (tok & mc)) << 4));
+          mma16816(oacc[2 * jj], pa0, pa2, cb4[0], cb4[1]);
+          mma16816(oacc[2 * jj + 1], pa0, pa2, cb4[2], cb4[3]);
+        }
+      }
+    }
+    __syncwarp();  // every lane is done with slot s (and read meta[s])
+    // refill this slot with tile i + SW; a tile's descriptor is read from the lane
+    // registers only when it is issued, so reloading the next 32 here is safe
+    const int nx = i + SW;
+    if (nx < my_tiles) {
+      if ((nx & 31) == 0) load_desc(nx);
+      issue(nx);
+    }
+  }
+  l_run += __shfl_xor_sync(kFull, l_run, 1);
+  l_run += __shfl_xor_sync(kFull, l_run, 2);
+  if (!ok) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
+
+  // merge the warps: each warp's (max, sum, acc[R]) per head -> one split result
+  constexpr int kOut = 2 + R;
+  float* mb = reinterpret_cast<float*>(smem);  // [kMmaWarps][G][kOut], reuses the rings
+  __syncthreads();
+  if (gr < G) {
+    float* dst = mb + ((size_t)w * G + gr) * kOut;
+    if (tq == 0) {
+      dst[0] = m_run;
+      dst[1] = l_run;
+    }
+#pragma unroll
+    for (int jj = 0; jj < NT; ++jj) {
+      dst[2 + 8 * jj + 2 * tq] = oacc[jj][0];
+      dst[3 + 8 * jj + 2 * tq] = oacc[jj][1];
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * R; idx += blockDim.x) {
+    const int hi = idx / R, dim = idx - hi * R;
+    float M = -INFINITY;
+#pragma unroll
+    for (int ww = 0; ww < kMmaWarps; ++ww) M = fmaxf(M, mb[((size_t)ww * G + hi) * kOut]);
+    float Ls = 0.f, As = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int ww = 0; ww < kMmaWarps; ++ww) {
+        const float* src = mb + ((size_t)ww * G + hi) * kOut;
+        const float f = exp2f(src[0] - M);  // 0 for a warp that saw nothing of this head
+        Ls += src[1] * f;
+        As += src[2 + dim] * f;
+      }
+    }
+    float* out = p.part + (((size_t)b * p.Hq + (size_t)g * G + hi) * p.nsplit + split) * (R + 2);
+    out[2 + dim] = As;
+    if (dim == 0) {
+      out[0] = M;
+      out[1] = Ls;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[bg], 1) == nsplit_active - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  merge_group_splits(p, b, g, G, R, nsplit_active, w, kMmaWarps, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -401,6 +699,42 @@ static cudaError_t launch_attn_g(const AttnParams& p, int G, int batch, cudaStre
   }
 }
 
+template <int D, int G, int NT>
+static cudaError_t launch_mma_t(const AttnParams& p, int batch, cudaStream_t st) {
+  const size_t stage = ((size_t)kTile * (D + NT * 8) * 2 + 127) & ~(size_t)127;
+  const size_t smem = (size_t)kMmaWarps * kMmaWarpStages * (stage + 8);
+  cudaError_t e = ensure_smem((const void*)attn_mma_kernel<D, G, NT>, smem);
+  if (e != cudaSuccess) return e;
+  attn_mma_kernel<D, G, NT><<<dim3(p.nsplit, p.Hkv, batch), 32 * kMmaWarps, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, int G>
+static cudaError_t launch_mma_r(const AttnParams& p, int batch, cudaStream_t st) {
+  switch (p.r / 8) {
+    case 2: return launch_mma_t<D, G, 2>(p, batch, st);
+    case 4: return launch_mma_t<D, G, 4>(p, batch, st);
+    case 6: return launch_mma_t<D, G, 6>(p, batch, st);
+    case 8: return launch_mma_t<D, G, 8>(p, batch, st);
+    case 10: return launch_mma_t<D, G, 10>(p, batch, st);
+    case 12: return launch_mma_t<D, G, 12>(p, batch, st);
+    case 14: return launch_mma_t<D, G, 14>(p, batch, st);
+    case 16: return launch_mma_t<D, G, 16>(p, batch, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D>
+static cudaError_t launch_mma_g(const AttnParams& p, int G, int batch, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_mma_r<D, 1>(p, batch, st);
+    case 2: return launch_mma_r<D, 2>(p, batch, st);
+    case 4: return launch_mma_r<D, 4>(p, batch, st);
+    case 8: return launch_mma_r<D, 8>(p, batch, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* scratch, int batch,
                                cudaStream_t st) {
   char* base = static_cast<char*>(scratch);
@@ -419,6 +753,8 @@ cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* 
                 a.Hq, a.Hkv, a.page, a.r, a.max_pages, a.num_phys, pl.umax, pl.tpp, pl.eps, pl.nsplit,
                 (float)(1.4426950408889634 / sqrt((double)a.d))};
   const int G = a.Hq / a.Hkv;
+  if (kc_swizzled(a.bf16, a.d, a.r))
+    return (a.d == 128) ? launch_mma_g<128>(ap, G, batch, st) : launch_mma_g<64>(ap, G, batch, st);
   if (a.bf16)
     return (a.d == 128) ? launch_attn_g<__nv_bfloat16, 128>(ap, G, batch, st)
                         : launch_attn_g<__nv_bfloat16, 64>(ap, G, batch, st);

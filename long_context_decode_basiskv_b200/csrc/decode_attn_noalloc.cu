@@ -65,7 +65,7 @@ extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
 
   // the same scratch basiskv_decode_attn takes from its workspace
   const DecodePlan plan = decode_plan(cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v, cfg->top_k,
-                                      batch, cache->max_pages);
+                                      batch, cache->max_pages, cfg->dtype == BASISKV_BF16, cfg->head_dim);
   if (plan.bytes > kNoAllocScratchBytes) {
     fprintf(stderr,
             "basiskv_decode_attn_noalloc: this shape needs %zu bytes of scratch, more than the "

@@ -78,7 +78,7 @@ struct DecodePlan {
   int nsplit;  // splits per (sequence, KV head)
   size_t uni_off, ucnt_off, cnt_off, part_off, bytes;
 };
-DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages);
+DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d);
 
 struct DecodeArgs {
   const void* q;
@@ -103,7 +103,9 @@ struct OutProjParams {
   int batch, K, hidden;
 };
 cudaError_t launch_out_proj_gemv(const OutProjParams& p, bool bf16, cudaStream_t st);
-bool out_proj_tc_supported(int K, int hidden, int batch);
+// bf16 shapes with K % 64 == 0 and hidden % 128 == 0 keep Gt in the blocked
+// tensor-core layout (see out_proj_tc.cu); every other shape uses [hidden][K].
+bool gt_blocked(int K, int hidden);
 cudaError_t launch_out_proj_tc(const float* o, const void* Gt, float* y, int32_t* err, int batch, int K, int hidden,
                                int num_sms, cudaStream_t st);
 
@@ -112,6 +114,7 @@ struct FuseParams {
   const void* W_O;
   void* Gt;
   int Hq, Hkv, d, r, hidden;
+  int blocked;  // write the tensor-core tile layout instead of [hidden][K]
 };
 cudaError_t launch_fuse(const FuseParams& p, bool bf16, cudaStream_t st);
 

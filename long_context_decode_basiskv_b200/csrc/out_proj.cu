@@ -82,7 +82,16 @@ __global__ void __launch_bounds__(128) fuse_kernel(FuseParams p) {
     for (int c = 0; c < kFuseCols && c0 + c < p.hidden; ++c) {
       double acc = 0.0;
       for (int j = 0; j < d; ++j) acc = fma((double)sB[i * ld + j], sW[j * kFuseCols + c], acc);
-      out[((size_t)(c0 + c) * p.Hq + h) * r + i] = Elem<T>::from_d(acc);
+      const int col = c0 + c, k = h * r + i;
+      size_t idx;
+      if (p.blocked) {
+        // tile (col / 128, k / 64); row col % 128 holds 8 chunks of 8, chunk j at j ^ (row % 8)
+        const int KC = p.Hq * r / 64, m = col & 127, kk = k & 63;
+        idx = (((size_t)(col >> 7) * KC + (k >> 6)) * 128 + m) * 64 + ((((kk >> 3) ^ (m & 7)) << 3) | (kk & 7));
+      } else {
+        idx = (size_t)col * p.Hq * r + k;
+      }
+      out[idx] = Elem<T>::from_d(acc);
     }
   }
 }

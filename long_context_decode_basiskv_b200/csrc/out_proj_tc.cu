@@ -7,8 +7,14 @@
 // both halves are multiplied into the same fp32 TMEM accumulator, so the
 // product keeps fp32-level accuracy with bf16 operands.
 //
-// Per CTA: warp 0 streams 128x64 tiles of Gt with 2-D TMA (128-byte swizzle,
-// no multicast) into a ring of 4-8 stages and one of its threads issues the
+// Gt is stored pre-tiled for this kernel (basiskv_fuse_out_factor writes it):
+// tile (m-tile, k-chunk) of 128 output columns x 64 latent dims is one
+// contiguous 16 KB block holding exactly the 128-byte-swizzled shared-memory
+// image the MMA reads, and the k-chunks of an m-tile are consecutive, so each
+// CTA streams one contiguous region with 1-D bulk copies.
+//
+// Per CTA: warp 0 streams the 16 KB tiles of Gt (cp.async.bulk, no multicast)
+// into a ring of 4-8 stages and one of its threads issues the
 // tcgen05.mma instructions, refilling each stage one iteration after its MMAs
 // were committed; warps 1-4 prefetch the matching slices of o with cp.async,
 // write them as swizzled bf16 hi/lo tiles into a matching ring and, at the
@@ -17,10 +23,7 @@
 // partial tiles are summed through distributed shared memory in a fixed
 // order (deterministic), each CTA writing a slice of the output rows.
 // HBM-bound: Gt is read once (16.8 MB for the 32K Llama-3-8B shape).
-#include <cuda.h>
 #include <stdio.h>
-
-#include <tuple>
 
 #include "kernels.cuh"
 
@@ -32,21 +35,14 @@ constexpr int kTcThreads = 160;  // warp 0: TMA + MMA; warps 1-4: o producers + 
 constexpr uint32_t kTcABytes = kTcM * kTcK * 2;
 
 struct OutProjTcParams {
-  const float* o;  // [B][K]
-  float* y;        // [B][hidden]
+  const __nv_bfloat16* Gt;  // blocked: [hidden/128][K/64] tiles of 128x64, each a swizzled 16 KB image
+  const float* o;           // [B][K]
+  float* y;                 // [B][hidden]
   int32_t* err;
   int batch, K, hidden, chunks_per_cta, ksplit;
 };
 
 // ---- PTX wrappers ------------------------------------------------------------
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
-          "r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -123,7 +119,7 @@ struct TcStages {
 
 template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    out_proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, OutProjTcParams p) {
+    out_proj_tc_kernel(OutProjTcParams p) {
   constexpr int S = TcStages<NB>::S;
   constexpr uint32_t kBBytes = NB * kTcK * 2;       // one of hi / lo per stage
   constexpr uint32_t kStageF32 = NB * kTcK * 4;     // fp32 staging of o per stage
@@ -176,9 +172,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     if (lane == 0 && nst > 0) {
       constexpr uint32_t idesc = idesc_bf16(kTcM, NB);
+      // this CTA's tiles of Gt are one contiguous run of 16 KB images
+      const __nv_bfloat16* gsrc = p.Gt + ((size_t)blockIdx.y * KC + ch0) * (kTcM * kTcK);
       for (int i = 0; i < min(S, nst); ++i) {
         mbar_arrive_expect_tx(&afull[i], kTcABytes);
-        tma_load_2d(sA + i * kTcABytes, &tmA, (ch0 + i) * kTcK, c0, &afull[i]);
+        bulk_g2s(sA + i * kTcABytes, gsrc + (size_t)i * (kTcM * kTcK), kTcABytes, &afull[i]);
       }
       for (int i = 0; i < nst; ++i) {
         const int s = i % S;
@@ -207,7 +205,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&afull[sp], kTcABytes);
-          tma_load_2d(sA + sp * kTcABytes, &tmA, (ch0 + ip + S) * kTcK, c0, &afull[sp]);
+          bulk_g2s(sA + sp * kTcABytes, gsrc + (size_t)(ip + S) * (kTcM * kTcK), kTcABytes, &afull[sp]);
         }
       }
       tc_commit(done);  // arrives when every MMA issued above has completed
@@ -315,64 +313,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // ---------------------------------------------------------------------------
 // host side: tensor map (cached per pointer/shape/device) and launch
 // ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-static cudaError_t gt_tensor_map(const void* Gt, int K, int hidden, CUtensorMap* out) {
-  struct Key {
-    int dev;
-    const void* ptr;
-    int K, hidden;
-    bool operator<(const Key& o) const {
-      return std::tie(dev, ptr, K, hidden) < std::tie(o.dev, o.ptr, o.K, o.hidden);
-    }
-  };
-  static std::mutex mu;
-  static std::map<Key, CUtensorMap> cache;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const Key key{dev, Gt, K, hidden};
-  std::lock_guard<std::mutex> lk(mu);
-  auto it = cache.find(key);
-  if (it != cache.end()) {
-    *out = it->second;
-    return cudaSuccess;
-  }
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return cudaErrorNotSupported;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)hidden};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kTcK, (cuuint32_t)kTcM};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Gt), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  if (cache.size() > 256) cache.clear();
-  cache[key] = map;
-  *out = map;
-  return cudaSuccess;
-}
-
-bool out_proj_tc_supported(int K, int hidden, int batch) {
-  return K % kTcK == 0 && hidden % kTcM == 0 && batch >= 1 && encode_fn() != nullptr;
-}
+bool gt_blocked(int K, int hidden) { return K % kTcK == 0 && hidden % kTcM == 0; }
 
 template <int NB>
 static size_t tc_smem_bytes() {
@@ -381,7 +322,7 @@ static size_t tc_smem_bytes() {
 }
 
 template <int NB>
-static cudaError_t launch_tc_nb(const CUtensorMap& map, OutProjTcParams p, int num_sms, cudaStream_t st) {
+static cudaError_t launch_tc_nb(OutProjTcParams p, int num_sms, cudaStream_t st) {
   const int mtiles = p.hidden / kTcM;
   const int bchunks = (p.batch + NB - 1) / NB;
   const int KC = p.K / kTcK;
@@ -404,21 +345,18 @@ static cudaError_t launch_tc_nb(const CUtensorMap& map, OutProjTcParams p, int n
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, out_proj_tc_kernel<NB>, map, p);
+  return cudaLaunchKernelEx(&cfg, out_proj_tc_kernel<NB>, p);
 }
 
 cudaError_t launch_out_proj_tc(const float* o, const void* Gt, float* y, int32_t* err, int batch, int K, int hidden,
                                int num_sms, cudaStream_t st) {
-  CUtensorMap map;
-  cudaError_t e = gt_tensor_map(Gt, K, hidden, &map);
-  if (e != cudaSuccess) return e;
-  OutProjTcParams p{o, y, err, batch, K, hidden, 0, 1};
+  OutProjTcParams p{static_cast<const __nv_bfloat16*>(Gt), o, y, err, batch, K, hidden, 0, 1};
   const int nb = batch <= 16 ? 16 : batch <= 32 ? 32 : batch <= 48 ? 48 : 64;
   switch (nb) {
-    case 16: return launch_tc_nb<16>(map, p, num_sms, st);
-    case 32: return launch_tc_nb<32>(map, p, num_sms, st);
-    case 48: return launch_tc_nb<48>(map, p, num_sms, st);
-    default: return launch_tc_nb<64>(map, p, num_sms, st);
+    case 16: return launch_tc_nb<16>(p, num_sms, st);
+    case 32: return launch_tc_nb<32>(p, num_sms, st);
+    case 48: return launch_tc_nb<48>(p, num_sms, st);
+    default: return launch_tc_nb<64>(p, num_sms, st);
   }
 }
 

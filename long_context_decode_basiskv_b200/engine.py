@@ -101,11 +101,25 @@ class DecodeEngine:
         self.out_proj(stream)
         return self.y
 
+    def kc_swizzled(self) -> bool:
+        """bf16 K and C pages are stored with 16-byte chunks XOR-swizzled per row."""
+        c = self.cfg
+        return c.dtype == torch.bfloat16 and c.head_dim % 16 == 0 and c.rank_v % 16 == 0
+
     def logical(self, tensor: torch.Tensor, b: int) -> torch.Tensor:
-        """Gather a per-page cache tensor [phys, Hkv, P, x] of sequence b into [Hkv, L, x]."""
+        """Gather a per-page cache tensor [phys, Hkv, P, x] of sequence b into [Hkv, L, x],
+        in token order and with the row swizzle of K and C pages undone."""
         L = self.case.lengths[b]
         n = -(-L // self.cfg.page_size)
         phys = self.cache.block_table[b, :n].long()
         t = tensor[phys]                       # [n, Hkv, P, x]
+        if self.kc_swizzled() and (tensor is self.cache.k_raw or tensor is self.cache.c_lat):
+            x = t.shape[-1]
+            chunks = x // 8
+            mask = 7 if chunks % 8 == 0 else 3 if chunks % 4 == 0 else 1 if chunks % 2 == 0 else 0
+            row = torch.arange(t.shape[2], device=t.device)[:, None]
+            src = ((torch.arange(chunks, device=t.device)[None, :] ^ (row & mask)) * 8)[..., None] \
+                + torch.arange(8, device=t.device)                          # [P, chunks, 8]
+            t = torch.gather(t, 3, src.reshape(1, 1, t.shape[2], x).expand_as(t))
         t = t.permute(1, 0, 2, 3).reshape(t.shape[1], n * self.cfg.page_size, -1)
         return t[:, :L]

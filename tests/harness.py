@@ -113,3 +113,22 @@ def assert_stored_equal(got, want, storage: str, what: str, max_frac: float = 1e
     assert not np.any(bad), f"{what}: {int(bad.sum())} values differ by more than 1 ulp"
     assert nd <= max(1, max_frac * got.size), f"{what}: {nd} of {got.size} values differ by 1 ulp"
     return nd
+
+
+def gt_plain(Gt: torch.Tensor, num_q_heads: int, rank_v: int, hidden: int) -> np.ndarray:
+    """Values of the fused factor as [hidden][Hq][r], whatever its storage layout.
+
+    bf16 shapes with K = Hq*r % 64 == 0 and hidden % 128 == 0 are stored in
+    128 x 64 tiles with XOR-swizzled 16-byte chunks (include/basiskv.h).
+    """
+    K = num_q_heads * rank_v
+    flat = Gt.detach().reshape(-1).cpu()
+    if Gt.dtype == torch.bfloat16 and K % 64 == 0 and hidden % 128 == 0:
+        t = flat.reshape(hidden // 128, K // 64, 128, 8, 8)          # [mt][kc][m][pos][e]
+        m = torch.arange(128)[:, None]
+        pos = torch.arange(8)[None, :] ^ (m % 8)                    # chunk j of row m sits at j ^ (m % 8)
+        t = t[:, :, m, pos, :]                                       # [mt][kc][m][j][e]
+        t = t.permute(0, 2, 1, 3, 4).reshape(hidden, K)
+    else:
+        t = flat.reshape(hidden, K)
+    return t.to(torch.float64).numpy().reshape(hidden, num_q_heads, rank_v)

@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from tests.harness import OracleCase, assert_close, assert_stored_equal, selection_ok, storage_of, to64
+from tests.harness import OracleCase, assert_close, assert_stored_equal, gt_plain, selection_ok, storage_of, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -127,7 +127,8 @@ def test_decode_attn_on_oracle_selection(run):
 
 
 def test_fused_factor_is_exact(run):
-    got = to64(run.eng.factors.Gt)                     # [hidden, Hq, r]
+    cfg = run.eng.cfg
+    got = gt_plain(run.eng.factors.Gt, cfg.num_q_heads, cfg.rank_v, cfg.hidden)   # [hidden, Hq, r]
     assert_stored_equal(got, run.oc.G.transpose(2, 0, 1), storage_of(run.wl), "Gt")
 
 
