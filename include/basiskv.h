@@ -74,6 +74,7 @@ typedef enum { BASISKV_F32 = 0, BASISKV_BF16 = 1 } basiskv_dtype;
 #define BASISKV_DEVERR_SELECTION 2     /* sel entry outside [0, pages of the sequence)       */
 #define BASISKV_DEVERR_SEQ_LEN 4       /* seq_len < n_new, or > max_pages * page_size         */
 #define BASISKV_DEVERR_TIMEOUT 8       /* an in-kernel wait on a bulk copy gave up (~1 s)     */
+#define BASISKV_DEVERR_WORKSPACE 16    /* a workspace counter was not zero: not zero-filled   */
 
 /*
  * Shapes.  Supported by this build: head_dim in {64, 128}; page_size in
@@ -166,7 +167,10 @@ BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basis
  * basiskv_append of the same step, which only rewrites the recent page: the
  * two may run concurrently on different streams.
  * workspace (device): at least basiskv_workspace_bytes(cfg, batch, max_pages)
- * bytes; contents need no initialisation and are clobbered.
+ * bytes, zero-filled once when it is allocated.  It holds per-call scratch
+ * plus small counters that every decode_attn call leaves at zero again, so no
+ * further clearing is needed between calls (a counter found out of range sets
+ * BASISKV_DEVERR_WORKSPACE).  Calls sharing one workspace must not overlap.
  */
 BASISKV_API basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache,
                              const void* q, int32_t batch, int32_t* sel, int32_t* sel_cnt,
@@ -203,8 +207,9 @@ BASISKV_API basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const 
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - Every call on a device shares the one array.  Calls that may overlap on
  *     the GPU (different streams without ordering) race and corrupt each
- *     other's results; order them.  The scratch needs no initialisation: each
- *     call writes every part of it that it reads.
+ *     other's results; order them.  The array is zero when the library loads
+ *     and every call leaves its counters at zero again, so it needs no
+ *     clearing.
  */
 BASISKV_API basiskv_status basiskv_decode_attn_noalloc(const basiskv_config* cfg,
                                                        const basiskv_cache* cache, const void* q,

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libbasiskv.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
-DEVERR_BLOCK_TABLE, DEVERR_SELECTION, DEVERR_SEQ_LEN, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_BLOCK_TABLE, DEVERR_SELECTION, DEVERR_SEQ_LEN, DEVERR_TIMEOUT, DEVERR_WORKSPACE = 1, 2, 4, 8, 16
 
 # every function include/basiskv.h declares
 SYMBOLS = [
@@ -179,7 +179,8 @@ def workspace_bytes(cfg: Config, batch: int, max_pages: int) -> int:
 
 
 def alloc_workspace(cfg: Config, batch: int, max_pages: int, device="cuda") -> torch.Tensor:
-    return torch.empty(max(workspace_bytes(cfg, batch, max_pages), 256), dtype=torch.uint8, device=device)
+    """A zero-filled workspace (the library keeps its counters at zero between calls)."""
+    return torch.zeros(max(workspace_bytes(cfg, batch, max_pages), 256), dtype=torch.uint8, device=device)
 
 
 def fuse_out_factor(cfg: Config, Bf: torch.Tensor, W_O: torch.Tensor, Gt: torch.Tensor, stream=None):

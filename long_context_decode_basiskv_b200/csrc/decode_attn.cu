@@ -7,12 +7,10 @@
 // restricted to the selected tokens, with the weights applied to the rank-r
 // Value latents instead of full-width values.
 //
-// Two launches:
-//  union  one CTA per (sequence, KV head): merges the G query heads'
-//         selections into one ascending page list with a G-bit head mask per
-//         page (a page chosen by several heads of a group is read once), and
-//         zeroes the group's split counter.
-//  attn   one CTA per (sequence, KV head, split of the union).  Warp 0 is the
+// One launch: one CTA per (sequence, KV head, split of the union).  Each CTA
+// first merges the G query heads' selections into the ascending union of
+// pages with a G-bit head mask per page (a page chosen by several heads of a
+// group is read once) and keeps its split's slice of it.  Warp 0 is the
 //         producer: its lanes hold the split's union entries (page, mask,
 //         physical page, valid tokens) and lane 0 streams 16-token tiles (raw
 //         K rows and C rows, each contiguous in the page block) into a ring of
@@ -55,10 +53,6 @@ DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, i
   pl.eps = (int)eps;
   pl.nsplit = (pl.umax + pl.eps - 1) / pl.eps;
   size_t off = 0;
-  pl.uni_off = off;
-  off += up256((size_t)batch * Hkv * pl.umax * 4);
-  pl.ucnt_off = off;
-  off += up256((size_t)batch * Hkv * 4);
   pl.cnt_off = off;
   off += up256((size_t)batch * Hkv * 4);
   pl.part_off = off;
@@ -68,24 +62,24 @@ DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, i
 }
 
 // ---------------------------------------------------------------------------
-// union of the group's selections
+// union of the group's selections, built by every CTA for its own split
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) union_kernel(UnionParams p) {
-  extern __shared__ __align__(16) uint32_t words[];  // [ceil(max_pages / 4)] byte masks
-  __shared__ int warp_tot[32];
-  __shared__ int s_cnt[8];
-  const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int G = p.Hq / p.Hkv;
+// All threads of the CTA call this.  It merges the G heads' selections of
+// (b, g) into per-page head masks in `words` (shared scratch of at least
+// ceil(n/4) words), ranks the selected pages in ascending order with a block
+// scan, stores the entries of rank e0 .. e0 + cap - 1 as page | mask << 24 in
+// `ent` (shared), and returns the union size U.
+__device__ int union_slice(const AttnParams& p, int b, int g, int G, int e0, int cap, uint32_t* words,
+                           uint32_t* ent, int* warp_tot, int* s_cnt) {
+  const int tid = threadIdx.x;
   const int row_len = p.top_k + 2;
   const size_t row0 = (size_t)b * p.Hq + (size_t)g * G;
   const int L = p.seq_len[b];
-  const int n = min((L + p.page - 1) / p.page, p.max_pages);
+  const int n = max(0, min((L + p.page - 1) / p.page, p.max_pages));
   const int nw = (n + 3) / 4;
-  if (tid == 0) p.cnt[(size_t)b * p.Hkv + g] = 0;
   if (tid < G) s_cnt[tid] = min(p.sel_cnt[row0 + tid], row_len);
   for (int i = tid; i < nw; i += blockDim.x) words[i] = 0u;
   __syncthreads();
-  // the G selection rows are contiguous: one flat pass, every load issued at once
   for (int i = tid; i < G * row_len; i += blockDim.x) {
     const int hi = i / row_len;
     if (i - hi * row_len >= s_cnt[hi]) continue;
@@ -103,18 +97,39 @@ __global__ void __launch_bounds__(256) union_kernel(UnionParams p) {
   for (int pg = lo; pg < hi; ++pg) c += ((words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu) ? 1 : 0;
   int tot;
   int pos = block_exclusive_scan(c, warp_tot, tot);
-  int32_t* out = p.uni + ((size_t)b * p.Hkv + g) * p.umax;
-  for (int pg = lo; pg < hi; ++pg) {
+  for (int pg = lo; pg < hi && pos < e0 + cap; ++pg) {
     const uint32_t m = (words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu;
     if (m) {
-      if (pos < p.umax) out[pos] = (int32_t)((uint32_t)pg | (m << 24));
+      if (pos >= e0) ent[pos - e0] = (uint32_t)pg | (m << 24);
       ++pos;
     }
   }
-  if (tid == 0) {
-    if (tot > p.umax) set_err(p.err, BASISKV_DEVERR_SELECTION);
-    p.ucnt[(size_t)b * p.Hkv + g] = min(tot, p.umax);
+  __syncthreads();
+  return tot;
+}
+
+// Offset of the split's entry list in dynamic shared memory: after the ring
+// (and its barriers), and after the page-mask scratch of union_slice.
+__host__ __device__ __forceinline__ size_t attn_ent_offset(size_t ring_bytes, int max_pages) {
+  const size_t masks = ((size_t)max_pages + 15) & ~(size_t)15;
+  return ((ring_bytes > masks ? ring_bytes : masks) + 15) & ~(size_t)15;
+}
+
+// After writing its split results, a CTA counts itself on the group's counter;
+// the last one of the group merges.  The merging CTA puts the counter back to
+// zero, so counters are zero between calls (the workspace is zero-filled once).
+__device__ __forceinline__ bool last_of_group(const AttnParams& p, size_t bg, int nsplit_active, int* s_last) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(&p.cnt[bg], 1);
+    if (prev >= nsplit_active) set_err(p.err, BASISKV_DEVERR_WORKSPACE);
+    *s_last = (prev == nsplit_active - 1);
   }
+  __syncthreads();
+  if (!*s_last) return false;
+  __threadfence();
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -196,8 +211,15 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.r;
   const size_t bg = (size_t)b * p.Hkv + g;
-  const int U = p.ucnt[bg];
   const int e0 = split * p.eps;
+  const uint32_t k_bytes = kTile * D * sizeof(T);
+  const uint32_t c_bytes = kTile * r * sizeof(T);
+  const uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
+  // shared memory: [ring | barriers] (page-mask scratch while the union is built) then the split's entries
+  uint32_t* ent = reinterpret_cast<uint32_t*>(smem + attn_ent_offset(kStages * stage_bytes + 2 * kStages * 8, p.max_pages));
+  __shared__ int warp_tot[32];
+  __shared__ int s_cnt[8];
+  const int U = union_slice(p, b, g, G, e0, p.eps, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
   const int nsplit_active = (U + p.eps - 1) / p.eps;
   if (e0 >= U) {
     // no work in this split; split 0 of an empty group still defines its output
@@ -208,10 +230,6 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   }
   const int nent = min(U, e0 + p.eps) - e0;
   const int ntiles = nent * p.tpp;
-
-  const uint32_t k_bytes = kTile * D * sizeof(T);
-  const uint32_t c_bytes = kTile * r * sizeof(T);
-  const uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * stage_bytes);
   uint64_t* empty = full + kStages;
 
@@ -230,7 +248,6 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
     const int L = p.seq_len[b];
     const int n = min((L + p.page - 1) / p.page, p.max_pages);
     const int last_valid = L - (n - 1) * p.page;
-    const int32_t* uni = p.uni + bg * p.umax;
     const T* kbase = static_cast<const T*>(p.k_raw);
     const T* cbase = static_cast<const T*>(p.c_lat);
     for (int cb = 0; cb < nent && ok; cb += 32) {
@@ -238,9 +255,9 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
       uint32_t my_mask = 0;
       int my_phys = -1, my_valid = 0;
       if (cb + lane < nent) {
-        const uint32_t ent = (uint32_t)uni[e0 + cb + lane];
-        const int pg = (int)(ent & 0xffffffu);
-        my_mask = ent >> 24;
+        const uint32_t en = ent[cb + lane];
+        const int pg = (int)(en & 0xffffffu);
+        my_mask = en >> 24;
         if (pg < n) {
           const int ph = p.block_table[(size_t)b * p.max_pages + pg];
           if (ph >= 0 && ph < p.num_phys) {
@@ -368,13 +385,9 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   if (!ok) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
 
   // the last CTA of the group to finish merges every split of its G heads
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[bg], 1) == nsplit_active - 1);
-  __syncthreads();
-  if (!s_last || warp == 0) return;
-  __threadfence();
-  merge_group_splits(p, b, g, G, r, nsplit_active, warp - 1, G, lane);
+  if (!last_of_group(p, bg, nsplit_active, &s_last)) return;
+  if (warp >= 1) merge_group_splits(p, b, g, G, r, nsplit_active, warp - 1, G, lane);
+  if (threadIdx.x == 0) p.cnt[bg] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -424,8 +437,16 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   uint32_t* meta = meta_all[w];
   const size_t bg = (size_t)b * p.Hkv + g;
-  const int U = p.ucnt[bg];
   const int e0 = split * p.eps;
+  constexpr uint32_t k_bytes = kTile * D * 2;
+  constexpr uint32_t c_bytes = kTile * R * 2;
+  constexpr uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
+  constexpr uint32_t ring_bytes = kMmaWarps * SW * (stage_bytes + 8);
+  // shared memory: [rings | barriers] (page-mask scratch while the union is built) then the split's entries
+  uint32_t* ent = reinterpret_cast<uint32_t*>(smem + attn_ent_offset(ring_bytes, p.max_pages));
+  __shared__ int warp_tot[32];
+  __shared__ int s_cnt[8];
+  const int U = union_slice(p, b, g, G, e0, p.eps, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
   const int nsplit_active = (U + p.eps - 1) / p.eps;
   if (e0 >= U) {
     if (split == 0 && U == 0)
@@ -436,9 +457,6 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
   const int nent = min(U, e0 + p.eps) - e0;
   const int ntiles = nent * p.tpp;
 
-  constexpr uint32_t k_bytes = kTile * D * 2;
-  constexpr uint32_t c_bytes = kTile * R * 2;
-  constexpr uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
   unsigned char* ring = smem + (size_t)w * SW * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kMmaWarps * SW * stage_bytes) + w * SW;
   if (lane == 0) {
@@ -450,7 +468,6 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
   const int L = p.seq_len[b];
   const int n = min((L + p.page - 1) / p.page, p.max_pages);
   const int last_valid = L - (n - 1) * p.page;
-  const int32_t* uni = p.uni + bg * p.umax;
   const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k_raw);
   const __nv_bfloat16* cbase = static_cast<const __nv_bfloat16*>(p.c_lat);
 
@@ -466,9 +483,9 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
     if (i < my_tiles) {
       const int t = w + kMmaWarps * i;
       const int e = t / p.tpp, sub = t - e * p.tpp;
-      const uint32_t ent = (uint32_t)uni[e0 + e];
-      const int pg = (int)(ent & 0xffffffu);
-      d_mask = ent >> 24;
+      const uint32_t en = ent[e];
+      const int pg = (int)(en & 0xffffffu);
+      d_mask = en >> 24;
       if (pg < n) {
         const int ph = p.block_table[(size_t)b * p.max_pages + pg];
         if (ph >= 0 && ph < p.num_phys) {
@@ -656,26 +673,22 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
       out[1] = Ls;
     }
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[bg], 1) == nsplit_active - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  if (!last_of_group(p, bg, nsplit_active, &s_last)) return;
   merge_group_splits(p, b, g, G, R, nsplit_active, w, kMmaWarps, lane);
+  if (threadIdx.x == 0) p.cnt[bg] = 0;
 }
 
 // ---------------------------------------------------------------------------
 // launch
 // ---------------------------------------------------------------------------
-size_t attn_smem_bytes(int d, int r, int esize) {
+size_t attn_smem_bytes(int d, int r, int esize, int max_pages, int eps) {
   const size_t stage = ((size_t)kTile * (d + r) * esize + 127) & ~(size_t)127;
-  return (size_t)kStages * stage + 2 * kStages * 8;
+  return attn_ent_offset((size_t)kStages * stage + 2 * kStages * 8, max_pages) + (size_t)eps * 4;
 }
 
 template <typename T, int D, int G, int CU>
 static cudaError_t launch_attn_t(const AttnParams& p, int batch, cudaStream_t st) {
-  const size_t smem = attn_smem_bytes(D, p.r, sizeof(T));
+  const size_t smem = attn_smem_bytes(D, p.r, sizeof(T), p.max_pages, p.eps);
   cudaError_t e = ensure_smem((const void*)attn_kernel<T, D, G, CU>, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nsplit, p.Hkv, batch);
@@ -702,7 +715,8 @@ static cudaError_t launch_attn_g(const AttnParams& p, int G, int batch, cudaStre
 template <int D, int G, int NT>
 static cudaError_t launch_mma_t(const AttnParams& p, int batch, cudaStream_t st) {
   const size_t stage = ((size_t)kTile * (D + NT * 8) * 2 + 127) & ~(size_t)127;
-  const size_t smem = (size_t)kMmaWarps * kMmaWarpStages * (stage + 8);
+  const size_t smem = attn_ent_offset((size_t)kMmaWarps * kMmaWarpStages * (stage + 8), p.max_pages) + (size_t)p.eps * 4;
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem((const void*)attn_mma_kernel<D, G, NT>, smem);
   if (e != cudaSuccess) return e;
   attn_mma_kernel<D, G, NT><<<dim3(p.nsplit, p.Hkv, batch), 32 * kMmaWarps, smem, st>>>(p);
@@ -738,21 +752,14 @@ static cudaError_t launch_mma_g(const AttnParams& p, int G, int batch, cudaStrea
 cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* scratch, int batch,
                                cudaStream_t st) {
   char* base = static_cast<char*>(scratch);
-  int32_t* uni = reinterpret_cast<int32_t*>(base + pl.uni_off);
-  int32_t* ucnt = reinterpret_cast<int32_t*>(base + pl.ucnt_off);
   int32_t* cnt = reinterpret_cast<int32_t*>(base + pl.cnt_off);
   float* part = reinterpret_cast<float*>(base + pl.part_off);
-  UnionParams up{a.sel, a.sel_cnt, a.seq_len, uni, ucnt, cnt, a.err, a.Hq, a.Hkv, a.page, a.max_pages, a.top_k,
-                 pl.umax};
-  const size_t usmem = ((size_t)a.max_pages + 3) / 4 * 4;
-  cudaError_t e = ensure_smem((const void*)union_kernel, usmem);
-  if (e != cudaSuccess) return e;
-  union_kernel<<<dim3(a.Hkv, batch), 256, usmem, st>>>(up);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  AttnParams ap{a.q, a.k_raw, a.c_lat, a.block_table, a.seq_len, uni, ucnt, cnt, part, a.o_lat, a.err,
-                a.Hq, a.Hkv, a.page, a.r, a.max_pages, a.num_phys, pl.umax, pl.tpp, pl.eps, pl.nsplit,
+  AttnParams ap{a.q, a.k_raw, a.c_lat, a.block_table, a.seq_len, a.sel, a.sel_cnt, cnt, part, a.o_lat, a.err,
+                a.Hq, a.Hkv, a.page, a.r, a.max_pages, a.num_phys, a.top_k, pl.umax, pl.tpp, pl.eps, pl.nsplit,
                 (float)(1.4426950408889634 / sqrt((double)a.d))};
+  cudaError_t e;
   const int G = a.Hq / a.Hkv;
+  (void)e;
   if (kc_swizzled(a.bf16, a.d, a.r))
     return (a.d == 128) ? launch_mma_g<128>(ap, G, batch, st) : launch_mma_g<64>(ap, G, batch, st);
   if (a.bf16)

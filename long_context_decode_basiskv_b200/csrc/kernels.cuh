@@ -43,29 +43,19 @@ struct SelectParams {
 cudaError_t launch_route(const ScoreParams& sp, const SelectParams& selp, int d, int G, bool bf16,
                          int num_sms, cudaStream_t st);
 
-struct UnionParams {
-  const int32_t* sel;
-  const int32_t* sel_cnt;
-  const int32_t* seq_len;
-  int32_t* uni;   // [B][Hkv][umax]  page | head mask << 24
-  int32_t* ucnt;  // [B][Hkv]
-  int32_t* cnt;   // [B][Hkv] finished-split counters (zeroed here)
-  int32_t* err;
-  int Hq, Hkv, page, max_pages, top_k, umax;
-};
 struct AttnParams {
   const void* q;
   const void* k_raw;
   const void* c_lat;
   const int32_t* block_table;
   const int32_t* seq_len;
-  const int32_t* uni;
-  const int32_t* ucnt;
-  int32_t* cnt;
+  const int32_t* sel;
+  const int32_t* sel_cnt;
+  int32_t* cnt;  // [B][Hkv] finished-split counters, zero between calls
   float* part;   // [B][Hq][nsplit][r + 2]
   float* o_lat;  // [B][Hq][r]
   int32_t* err;
-  int Hq, Hkv, page, r, max_pages, num_phys, umax, tpp, eps, nsplit;
+  int Hq, Hkv, page, r, max_pages, num_phys, top_k, umax, tpp, eps, nsplit;
   float qscale;  // log2(e) / sqrt(d)
 };
 
@@ -76,7 +66,7 @@ struct DecodePlan {
   int tpp;     // 16-token tiles per page
   int eps;     // union pages per split
   int nsplit;  // splits per (sequence, KV head)
-  size_t uni_off, ucnt_off, cnt_off, part_off, bytes;
+  size_t cnt_off, part_off, bytes;
 };
 DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d);
 
