@@ -130,14 +130,12 @@ basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cac
   if (!aligned16(q) || (scores && !aligned16(scores))) return BASISKV_ERR_INVALID_ARG;
   const Workspace w = layout(cfg, batch, cache->max_pages);
   if (!ws || ws_bytes < w.total || !aligned16(ws)) return BASISKV_ERR_WORKSPACE;
-  float* sc = scores ? scores : reinterpret_cast<float*>(static_cast<char*>(ws) + w.scores);
-  ScoreParams sp{q, cache->summary, cache->block_table, cache->seq_len, sc, err_flag,
+  char* wsb = static_cast<char*>(ws);
+  float* sc = scores ? scores : reinterpret_cast<float*>(wsb + w.scores);
+  RouteParams rp{q, cache->summary, cache->block_table, cache->seq_len, sc, sel, sel_cnt, err_flag,
                  batch, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cache->max_pages,
-                 cache->num_phys_pages, (cache->max_pages + 7) / 8, scores ? 1 : 0};
-  SelectParams selp{sc, cache->seq_len, sel, sel_cnt, cfg->num_q_heads, cfg->page_size,
-                    cache->max_pages, cfg->top_k};
-  return cuda_status(launch_route(sp, selp, cfg->head_dim, cfg->num_q_heads / cfg->num_kv_heads,
-                                  cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream));
+                 cache->num_phys_pages, cfg->top_k, scores ? 1 : 0};
+  return cuda_status(launch_route(rp, cfg->head_dim, cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream));
 }
 
 basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,

@@ -22,26 +22,19 @@ struct AppendParams {
 };
 cudaError_t launch_append(const AppendParams& p, bool bf16, cudaStream_t st);
 
-struct ScoreParams {
+struct RouteParams {
   const void* q;
   const float* summary;
   const int32_t* block_table;
   const int32_t* seq_len;
-  float* scores;
+  float* scores;    // [B][Hq][max_pages]
+  int32_t* sel;     // [B][Hq][top_k + 2]
+  int32_t* sel_cnt; // [B][Hq]
   int32_t* err;
-  int batch, Hq, Hkv, page, max_pages, num_phys;
-  int page_batches;
-  int all_pages;  // 0: skip the sink and recent pages (always kept; their scores are not needed)
+  int batch, Hq, Hkv, page, max_pages, num_phys, top_k;
+  int all_pages;    // 0: skip the sink and recent pages (always kept; their scores are not needed)
 };
-struct SelectParams {
-  const float* scores;
-  const int32_t* seq_len;
-  int32_t* sel;
-  int32_t* sel_cnt;
-  int Hq, page, max_pages, top_k;
-};
-cudaError_t launch_route(const ScoreParams& sp, const SelectParams& selp, int d, int G, bool bf16,
-                         int num_sms, cudaStream_t st);
+cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st);
 
 struct AttnParams {
   const void* q;

@@ -5,78 +5,89 @@
 // keeps its mean predicted key S_p, each query head scores all pages with
 // q_h . S_p and keeps the top-k, plus the sink page 0 and the recent page.
 //
-// Kernel 1 (score): streams the fp32 summaries once.  A warp takes 8 pages of
-// one (sequence, KV head); each lane loads its d/32 dimensions of the 8
-// summary rows (8 independent 16-byte loads in flight per lane), forms the
-// partial dot products with all G query heads of the group, and one
-// transpose-reduction leaves one (page, head) score per lane.  The summary of
-// a page is read once for the whole GQA group.  HBM-bound.
+// Kernel 1 (score) streams the fp32 summaries once; HBM-bound.  Grid (chunk,
+// KV head g, sequence b): CTA c scores pages [c * 256, c * 256 + 256) of
+// (b, g) for the G query heads of the group, warp w the 32 pages starting at
+// c * 256 + w * 32 in four 8-page items: one coalesced block-table load per
+// warp; per item one 16-byte summary load per lane and page, the G partial dot
+// products against the query rows (held in registers), and one
+// transpose-reduction that leaves one (page, head) score per lane.  The
+// summary of a page is read once for the whole GQA group.  The grid is one
+// resident wave (<= 64 registers, 4 CTAs per SM).
 //
-// Kernel 2 (select): one CTA per (sequence, query head) finds T, the exact
-// k-th largest score: a 256-bucket histogram over the linear score range (a
-// monotone map, so whole buckets above the boundary bucket are kept) narrows
-// the search to the boundary bucket, refined up to three times, whose few
-// scores are ranked exactly.  Pages scoring above T are kept, ties at T go to
-// the lowest page indices, and a block scan compacts the kept pages (plus the
-// sink and recent pages) in ascending order.
+// Kernel 2 (select), one CTA per (sequence, query head), exact:
+//   * each thread holds the scores of up to KPT consecutive pages as
+//     order-preserving 32-bit keys (NaN lowest, -0 == +0) in registers;
+//   * T, the k-th largest key of pages 1..n-2, is found bit by bit from the
+//     top: a bit is set when at least k keys are >= the prefix with it set (a
+//     block-wide count per bit); when exactly k keys are >= the prefix, those
+//     k are the answer and there are no ties to break;
+//   * pages with key > T are kept, and of the keys equal to T the ones with
+//     the lowest page indices; two block scans (ties, kept pages) give every
+//     thread its output positions, so sel is written in ascending page order.
+// The result is the same as sorting by (score descending, page ascending).
 #include "kernels.cuh"
 
 namespace bkv {
 
-
-
+constexpr int kPagesPerWarp = 8;   // pages per warp item of the score kernel
 constexpr int kScoreThreads = 256;
-constexpr int kPagesPerWarp = 8;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kScoreWarpPages = 32;
+constexpr int kScoreCtaPages = kScoreWarps * kScoreWarpPages;
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_kernel(RouteParams p) {
   constexpr int DPL = D / 32;
   constexpr int N = kPagesPerWarp * G;
-  const int lane = threadIdx.x & 31;
-  const int warps_total = gridDim.x * (blockDim.x / 32);
-  const int wid = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const long long items = (long long)p.batch * p.Hkv * p.page_batches;
+  __shared__ __align__(16) float sq[G * D];
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int L = p.seq_len[b];
+  int n = (L + p.page - 1) / p.page;
+  if (n > p.max_pages) {
+    if (c == 0 && tid == 0) set_err(p.err, BASISKV_DEVERR_SEQ_LEN);
+    n = p.max_pages;
+  }
+  const int pw0 = c * kScoreCtaPages + warp * kScoreWarpPages;
+  if (c * kScoreCtaPages >= n) return;  // the whole CTA is past the last page
+  const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;
+  const T* qb = static_cast<const T*>(p.q) + qrow * D;
+  for (int i = tid; i < G * D; i += kScoreThreads) sq[i] = Elem<T>::to_f(qb[i]);
 
-  for (long long it = wid; it < items; it += warps_total) {
-    const int pb = (int)(it % p.page_batches);
-    const int bg = (int)(it / p.page_batches);
-    const int g = bg % p.Hkv, b = bg / p.Hkv;
-    const int L = p.seq_len[b];
-    int n = (L + p.page - 1) / p.page;
-    if (n > p.max_pages) {
-      if (pb == 0 && lane == 0) set_err(p.err, BASISKV_DEVERR_SEQ_LEN);
-      n = p.max_pages;
-    }
-    const int p0 = pb * kPagesPerWarp;
-    if (p0 >= n) continue;
-
-    float qf[G][DPL];
-    const T* qb = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
-#pragma unroll
-    for (int hi = 0; hi < G; ++hi)
-#pragma unroll
-      for (int u = 0; u < DPL; ++u) qf[hi][u] = Elem<T>::to_f(qb[hi * D + lane * DPL + u]);
-
-    int my_phys = -1;
-    const int pl = p0 + lane;
-    if (lane < kPagesPerWarp && pl < n && (p.all_pages || (pl != 0 && pl != n - 1))) {
-      my_phys = p.block_table[(size_t)b * p.max_pages + p0 + lane];
+  int my_phys = -1;  // -1: not scored, -2: bad block-table entry
+  {
+    const int pl = pw0 + lane;
+    if (pl < n && (p.all_pages || (pl != 0 && pl != n - 1))) {
+      my_phys = p.block_table[(size_t)b * p.max_pages + pl];
       if (my_phys < 0 || my_phys >= p.num_phys) {
         set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
         my_phys = -2;
       }
     }
+  }
+  __syncthreads();  // sq
+  float qf[G][DPL];  // this lane's dimensions of the G query rows
+#pragma unroll
+  for (int hi = 0; hi < G; ++hi)
+#pragma unroll
+    for (int u = 0; u < DPL; ++u) qf[hi][u] = sq[hi * D + lane * DPL + u];
+  float* outb = p.scores + qrow * p.max_pages;
+#pragma unroll 1
+  for (int i0 = 0; i0 < kScoreWarpPages; i0 += kPagesPerWarp) {
+    const int p0 = pw0 + i0;
+    if (p0 >= n) break;
     float sv[kPagesPerWarp][DPL];
 #pragma unroll
     for (int i = 0; i < kPagesPerWarp; ++i) {
-      const int ph = __shfl_sync(kFull, my_phys, i);
+      const int ph = __shfl_sync(kFull, my_phys, i0 + i);
       if (ph >= 0) {
-        const float* row = p.summary + ((size_t)ph * p.Hkv + g) * D + lane * DPL;
+        const float* rowp = p.summary + ((size_t)ph * p.Hkv + g) * D + lane * DPL;
         if constexpr (DPL == 4) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(row));
+          const float4 v = __ldg(reinterpret_cast<const float4*>(rowp));
           sv[i][0] = v.x; sv[i][1] = v.y; sv[i][2] = v.z; sv[i][3] = v.w;
         } else {
-          const float2 v = __ldg(reinterpret_cast<const float2*>(row));
+          const float2 v = __ldg(reinterpret_cast<const float2*>(rowp));
           sv[i][0] = v.x; sv[i][1] = v.y;
         }
       } else {
@@ -95,13 +106,12 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
         part[i * G + hi] = a;
       }
     transpose_reduce<N>(part, lane);
-
-    float* out = p.scores + ((size_t)b * p.Hq + (size_t)g * G) * p.max_pages + p0;
+    float* out = outb + p0;
     if constexpr (N <= 32) {
       constexpr int kDup = 32 / N;
       const int idx = lane / kDup;
       const int i = idx / G, hi = idx % G;
-      const int ph = __shfl_sync(kFull, my_phys, i);
+      const int ph = __shfl_sync(kFull, my_phys, i0 + i);
       if ((lane % kDup) == 0 && p0 + i < n && ph != -1)
         out[(size_t)hi * p.max_pages + i] = (ph == -2) ? -INFINITY : part[0];
     } else {
@@ -109,7 +119,7 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
       for (int j = 0; j < 2; ++j) {
         const int idx = 2 * lane + j;
         const int i = idx / G, hi = idx % G;
-        const int ph = __shfl_sync(kFull, my_phys, i);
+        const int ph = __shfl_sync(kFull, my_phys, i0 + i);
         if (p0 + i < n && ph != -1) out[(size_t)hi * p.max_pages + i] = (ph == -2) ? -INFINITY : part[j];
       }
     }
@@ -117,9 +127,116 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreParams 
 }
 
 // ---------------------------------------------------------------------------
-// selection
+// selection with the keys in registers
 // ---------------------------------------------------------------------------
 constexpr int kSelectThreads = 256;
+constexpr int kSelectWarps = kSelectThreads / 32;
+
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 0u;  // NaN: below every score
+  if (v == 0.f) v = 0.f;  // -0 ties with +0
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Sum of one int per thread over the block.  `red` is shared scratch of
+// 2 * kSelectWarps ints used alternately (`phase` flips it), so one barrier
+// per call suffices.
+__device__ __forceinline__ int block_total(int v, int* red, int& phase) {
+  v = (int)__reduce_add_sync(kFull, (unsigned)v);
+  int* slot = red + (phase & 1) * kSelectWarps;
+  ++phase;
+  if ((threadIdx.x & 31) == 0) slot[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int t = 0;
+#pragma unroll
+  for (int w = 0; w < kSelectWarps; ++w) t += slot[w];
+  return t;
+}
+
+template <int KPT>
+__global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
+  __shared__ int red[2 * kSelectWarps];
+  __shared__ int warp_tot[32];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int L = p.seq_len[b];
+  const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
+  const int kk = p.top_k;
+  const size_t row = (size_t)b * p.Hq + h;
+  int32_t* out = p.sel + row * (kk + 2);
+  if (n <= kk + 2) {
+    for (int i = tid; i < kk + 2; i += kSelectThreads) out[i] = (i < n) ? i : -1;
+    if (tid == 0) p.sel_cnt[row] = n;
+    return;
+  }
+  // thread t holds pages [t * KPT, t * KPT + KPT)
+  const float* sc = p.scores + row * p.max_pages;
+  const int p0 = tid * KPT;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int pg = p0 + j;
+    key[j] = (pg >= 1 && pg <= n - 2) ? order_key(sc[pg]) : 0u;  // 0: not a candidate
+  }
+  auto count_ge = [&](uint32_t t) {
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) c += key[j] >= t;
+    return c;
+  };
+  int phase = 0;
+  uint32_t T = 0;
+  bool exact = false;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    const int c = block_total(count_ge(cand), red, phase);
+    if (c >= kk) {
+      T = cand;
+      if (c == kk) {
+        exact = true;
+        break;
+      }
+    }
+  }
+  int keep_eq;
+  if (exact) {
+    T -= 1;  // keep key > T; no ties (at least one bit of T was set)
+    keep_eq = 0;
+  } else {
+    keep_eq = kk - ((T == 0xffffffffu) ? 0 : block_total(count_ge(T + 1), red, phase));
+  }
+  // ties at T before this thread's pages (page order), then kept pages before them
+  int ties = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) ties += key[j] != 0u && key[j] == T;
+  int tot;
+  const int tie0 = block_exclusive_scan(ties, warp_tot, tot);
+  bool take[KPT];
+  int kept = 0;
+  {
+    int tr = tie0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int pg = p0 + j;
+      const bool tie = key[j] != 0u && key[j] == T;
+      take[j] = pg == 0 || pg == n - 1 || key[j] > T || (tie && tr < keep_eq);
+      take[j] = take[j] && pg < n;
+      tr += tie;
+      kept += take[j];
+    }
+  }
+  int total;
+  int pos = block_exclusive_scan(kept, warp_tot, total);
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if (take[j]) out[pos++] = p0 + j;
+  for (int i = total + tid; i < kk + 2; i += kSelectThreads) out[i] = -1;
+  if (tid == 0) p.sel_cnt[row] = total;
+}
+
+// ---------------------------------------------------------------------------
+// selection for block tables wider than the register-key kernel handles
+// ---------------------------------------------------------------------------
 constexpr int kCandCap = 512;  // boundary candidates ranked exactly in shared memory
 constexpr int kLevels = 3;     // histogram refinements of the boundary bucket
 
@@ -159,10 +276,14 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
   return t;
 }
 
-// One CTA per (sequence, query head).  Finds T, the k-th largest score of
-// pages 1..n-2, and how many pages scoring exactly T are kept (the lowest
-// indices), then writes the kept pages plus 0 and n-1 in ascending order.
-__global__ void __launch_bounds__(kSelectThreads) route_select_kernel(SelectParams p) {
+// One CTA per (sequence, query head), scores staged in shared memory.  A
+// 256-bucket histogram over the linear score range (a monotone map, so whole
+// buckets above the boundary bucket are kept) narrows the search to the
+// boundary bucket, refined up to three times; its few scores are ranked
+// exactly.  Finds T, the k-th largest score of pages 1..n-2, and how many pages
+// scoring exactly T are kept (the lowest indices), then writes the kept pages
+// plus 0 and n-1 in ascending order.
+__global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(RouteParams p) {
   extern __shared__ __align__(16) float ssc[];  // [max_pages] scores of this head
   __shared__ int hist[256];
   __shared__ int warp_tot[32];
@@ -343,11 +464,14 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(SelectPara
   if (tid == 0) p.sel_cnt[row] = tot;
 }
 
+
 // ---------------------------------------------------------------------------
 // launch
 // ---------------------------------------------------------------------------
 template <typename T, int D>
-static cudaError_t launch_score_g(const ScoreParams& p, int G, int grid, cudaStream_t st) {
+static cudaError_t launch_score_g(const RouteParams& p, int G, cudaStream_t st) {
+  const int nchunk = (p.max_pages + kScoreCtaPages - 1) / kScoreCtaPages;
+  const dim3 grid(nchunk, p.Hkv, p.batch);
   switch (G) {
     case 1: route_score_kernel<T, D, 1><<<grid, kScoreThreads, 0, st>>>(p); break;
     case 2: route_score_kernel<T, D, 2><<<grid, kScoreThreads, 0, st>>>(p); break;
@@ -358,28 +482,27 @@ static cudaError_t launch_score_g(const ScoreParams& p, int G, int grid, cudaStr
   return cudaGetLastError();
 }
 
-cudaError_t launch_route(const ScoreParams& sp, const SelectParams& selp, int d, int G, bool bf16,
-                         int num_sms, cudaStream_t st) {
-  const long long items = (long long)sp.batch * sp.Hkv * sp.page_batches;
-  const long long warps = (items + 0);
-  long long blocks = (warps + (kScoreThreads / 32) - 1) / (kScoreThreads / 32);
-  const long long cap = (long long)num_sms * (2048 / kScoreThreads);
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
+cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st) {
+  (void)num_sms;
+  const int G = p.Hq / p.Hkv;
   cudaError_t e;
-  if (bf16) {
-    e = (d == 128) ? launch_score_g<__nv_bfloat16, 128>(sp, G, (int)blocks, st)
-                   : launch_score_g<__nv_bfloat16, 64>(sp, G, (int)blocks, st);
+  if (bf16)
+    e = (d == 128) ? launch_score_g<__nv_bfloat16, 128>(p, G, st) : launch_score_g<__nv_bfloat16, 64>(p, G, st);
+  else
+    e = (d == 128) ? launch_score_g<float, 128>(p, G, st) : launch_score_g<float, 64>(p, G, st);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(p.Hq, p.batch);
+  if (p.max_pages <= kSelectThreads * 8) {
+    route_select_kernel<8><<<grid, kSelectThreads, 0, st>>>(p);
+  } else if (p.max_pages <= kSelectThreads * 16) {
+    route_select_kernel<16><<<grid, kSelectThreads, 0, st>>>(p);
+  } else if (p.max_pages <= kSelectThreads * 32) {
+    route_select_kernel<32><<<grid, kSelectThreads, 0, st>>>(p);
   } else {
-    e = (d == 128) ? launch_score_g<float, 128>(sp, G, (int)blocks, st)
-                   : launch_score_g<float, 64>(sp, G, (int)blocks, st);
+    const size_t smem = (size_t)p.max_pages * sizeof(float);
+    if ((e = ensure_smem((const void*)route_select_hist_kernel, smem)) != cudaSuccess) return e;
+    route_select_hist_kernel<<<grid, kSelectThreads, smem, st>>>(p);
   }
-  if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)sp.max_pages * sizeof(float);
-  e = ensure_smem((const void*)route_select_kernel, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(sp.Hq, sp.batch);
-  route_select_kernel<<<grid, kSelectThreads, smem, st>>>(selp);
   return cudaGetLastError();
 }
 

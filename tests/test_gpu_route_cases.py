@@ -75,3 +75,37 @@ def test_selection_on_crafted_scores(eng, kind):
             got = sel[b, h, :cnt[b, h]]
             np.testing.assert_array_equal(got, wants[b], err_msg=f"{kind} b={b} h={h}")
             assert np.all(sel[b, h, cnt[b, h]:] == -1)
+
+
+@pytest.mark.parametrize("width", [6000, 8192 + 40])
+def test_wide_block_tables(eng, width):
+    """Wider block tables select with other kernel instances (32 register keys
+    per thread up to 8192 pages, the shared-memory histogram kernel beyond);
+    they must select exactly the pages of the narrow table."""
+    rng = np.random.default_rng(7)
+    cfg, cache = eng.cfg, eng.cache
+    B = cache.batch
+    for b in range(B):
+        n = -(-eng.case.lengths[b] // cfg.page_size)
+        S = np.zeros((n, cfg.head_dim), dtype=np.float32)
+        S[:, 0] = rng.integers(-50, 50, size=n)
+        phys = cache.block_table[b, :n].long()
+        for g in range(cfg.num_kv_heads):
+            cache.summary[phys, g] = torch.from_numpy(S).cuda()
+    eng.err.zero_()
+    bk.route(cfg, cache, eng.q, eng.sel, eng.sel_cnt, eng.ws, eng.err)
+    torch.cuda.synchronize()
+    ref_sel, ref_cnt = eng.sel.clone(), eng.sel_cnt.clone()
+
+    wide = bk.PagedCache.__new__(bk.PagedCache)
+    wide.__dict__.update(cache.__dict__)
+    bt = torch.full((B, width), -1, dtype=torch.int32, device="cuda")
+    bt[:, :cache.max_pages] = cache.block_table
+    wide.block_table = bt
+    ws = bk.alloc_workspace(cfg, B, width, device="cuda")
+    eng.sel.fill_(-7)
+    bk.route(cfg, wide, eng.q, eng.sel, eng.sel_cnt, ws, eng.err)
+    torch.cuda.synchronize()
+    assert int(eng.err.item()) == 0
+    assert torch.equal(eng.sel, ref_sel)
+    assert torch.equal(eng.sel_cnt, ref_cnt)
