@@ -6,10 +6,13 @@
 One step = one decode step of one attention layer for every sequence of the
 batch: append (latent + residual + page summary), route (page scores + top-k),
 decode_attn (exact attention on the routed pages), out_proj (fused factor).
-The metric is decode tokens/s per layer (batch / step time).  Each C-ABI call
-is captured once into its own CUDA graph; a timed step replays the four graphs
-with CUDA events between them on the launching stream.  L2 is flushed between
-steps by reading a 256 MiB buffer (outside the events).
+The metric is decode tokens/s per layer (batch / step time).  The whole step
+(append on a forked stream concurrently with route, then decode_attn and
+out_proj) is captured once into a CUDA graph; a timed step is one replay
+bracketed by CUDA events on the launching stream.  A second pass replays one
+graph per phase, with events between them, for the per-kernel breakdown and
+the roofline of the attention kernel.  L2 is flushed before every step by
+reading a 256 MiB buffer (outside the events).
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent
 replica on its own sequences (weak scaling; the path has no exchange step).
@@ -39,7 +42,10 @@ from long_context_decode_basiskv_b200.workloads import WORKLOADS, make_case  # n
 METRIC = "decode tokens/s per layer on 1 B200; route+attn HBM GB/s vs ~8 TB/s roofline"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNELS_PER_STEP = 7  # append 1, route 2 (score, select), decode_attn 3 (union, attn, combine), out_proj 1
+# kernels one decode step launches: append_decode, route_score, route_select,
+# the sparse attention kernel (union slice, attention and split merge in one
+# launch) and the out-projection kernel
+KERNELS_PER_STEP = 5
 
 
 def parse():
@@ -74,6 +80,13 @@ def init_dist(world, backend):
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
+
+
+def replica_workload(wl, rank: int, world: int):
+    """Weak scaling: every rank decodes its own sequences (a different seed per rank)."""
+    if world > 1:
+        return dataclasses.replace(wl, seed=wl.seed + 1000 * rank)
+    return wl
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -246,9 +259,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
-    wl = WORKLOADS[args.workload]
-    if world > 1:
-        wl = dataclasses.replace(wl, seed=wl.seed + 1000 * rank)   # different sequences per replica
+    wl = replica_workload(WORKLOADS[args.workload], rank, world)
     case = make_case(wl, dev)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
@@ -259,9 +270,9 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"device error flag {int(eng.err.item())}")
     nbytes = algorithmic_bytes(eng)
 
-    # one CUDA graph per phase: append || route (forked streams), decode_attn, out_proj
+    # the whole step as one CUDA graph, and one graph per phase for the breakdown
     graphs = {}
-    for name, fn in [("append_route", eng.append_route), ("decode_attn", eng.decode_attn),
+    for name, fn in [("step", eng.step), ("append_route", eng.append_route), ("decode_attn", eng.decode_attn),
                      ("out_proj", eng.out_proj)]:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
@@ -272,15 +283,15 @@ def run_ours(args, world, rank, local):
     flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
     sink = torch.zeros((), dtype=torch.float32, device=dev)
 
-    def run_steps(n, record):
+    def run_steps(n, record, phases):
         evs = []
         with torch.cuda.stream(stream):
             for _ in range(n):
                 torch.sum(flush, dim=0, out=sink)
-                e = [torch.cuda.Event(enable_timing=True) for _ in range(len(order) + 1)] if record else None
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] if record else None
                 if record:
                     e[0].record(stream)
-                for i, name in enumerate(order):
+                for i, name in enumerate(phases):
                     graphs[name].replay()
                     if record:
                         e[i + 1].record(stream)
@@ -288,17 +299,21 @@ def run_ours(args, world, rank, local):
                     evs.append(e)
         return evs
 
-    run_steps(args.warmup, False)
+    run_steps(args.warmup, False, ["step"])
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        evs = run_steps(args.steps, True)
+        evs = run_steps(args.steps, True, ["step"])
         torch.cuda.synchronize()
     barrier(world)
-    per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, name in enumerate(order)}
-    step_ms = [ev[0].elapsed_time(ev[-1]) for ev in evs]
+    step_ms = [ev[0].elapsed_time(ev[1]) for ev in evs]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
+    # per-phase breakdown (separate pass; not part of the headline number)
+    run_steps(max(3, args.warmup), False, order)
+    evs = run_steps(min(args.steps, 100), True, order)
+    torch.cuda.synchronize()
+    per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, name in enumerate(order)}
     ms_per_step = total_ms / args.steps
     value = world * wl.batch * args.steps / (total_ms / 1e3)
 
@@ -308,7 +323,7 @@ def run_ours(args, world, rank, local):
     ra_gbs = (nbytes["route"] + nbytes["decode_attn"]) / ((mean["append_route"] + mean["decode_attn"]) * 1e-3) / 1e9
     traffic_rec = profiled_traffic("decode_attn.cu")
     roofline = {
-        "kernel": "basiskv_decode_attn (union + attn + combine launches)",
+        "kernel": "basiskv_decode_attn (one launch: union slice, attention, split merge)",
         "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
         "frac": round(attn_gbs / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
         "algorithmic_bytes": nbytes["decode_attn"],
@@ -371,7 +386,7 @@ def run_ours(args, world, rank, local):
                        "page_size": wl.page_size, "rank_v": wl.rank_v, "rank_k": wl.rank_k,
                        "top_k": wl.top_k, "hidden": wl.hidden, "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps (read of a 256 MiB buffer)",
-                       "timing": "CUDA graphs per phase (append || route on forked streams, decode_attn, out_proj), CUDA events between them; route+attn GB/s counts the append || route phase time"},
+                       "timing": "one CUDA graph per step (append || route on forked streams, decode_attn, out_proj), CUDA events around each replay; kernels_us from per-phase graphs in a separate pass; route+attn GB/s counts the append || route phase time"},
             "kernels_us": {k: round(v * 1e3, 2) for k, v in mean.items()},
             "algorithmic_bytes": nbytes,
             "route_attn_gbs": round(ra_gbs, 1),
