@@ -64,7 +64,7 @@ static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 static Workspace layout(const basiskv_config* c, int batch, int max_pages) {
   Workspace w{};
   w.plan = decode_plan(c->num_q_heads, c->num_kv_heads, c->page_size, c->rank_v, c->top_k, batch, max_pages,
-                       c->dtype == BASISKV_BF16, c->head_dim);
+                       c->dtype == BASISKV_BF16, c->head_dim, num_sms());
   w.scores = 0;
   w.decode = up256((size_t)batch * c->num_q_heads * max_pages * 4);
   w.total = w.decode + w.plan.bytes;

@@ -30,28 +30,32 @@ namespace bkv {
 
 constexpr int kTile = 16;           // tokens per tile
 constexpr int kStages = 4;          // ring depth per CTA
-constexpr int kTargetCtas = 888;    // one wave of attn CTAs on a B200 (148 SMs x 6)
+constexpr int kCoreCtasPerSm = 6;   // resident CTAs per SM of the CUDA-core attention kernel
+constexpr int kMmaCtasPerSm = 3;    // ... and of the tensor-core one (registers and shared memory)
 
 // ---------------------------------------------------------------------------
-// plan: tiles per split and scratch layout (independent of the device)
+// plan: splits per (sequence, KV head) and the scratch layout
 // ---------------------------------------------------------------------------
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d) {
+// Every (sequence, KV head) group gets the same number of splits, as many as
+// one resident wave of the kernel holds (at least one); each split takes an
+// equal share of its group's union at run time, at most eps pages.
+DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d,
+                       int num_sms) {
   DecodePlan pl{};
-  const int target = kc_swizzled(bf16, d, r) ? 444 : kTargetCtas;  // CTAs per wave of the kernel that runs
+  const long long slots = (long long)num_sms * (kc_swizzled(bf16, d, r) ? kMmaCtasPerSm : kCoreCtasPerSm);
   const int G = Hq / Hkv;
   long long um = (long long)G * (top_k + 2);
   if (um > max_pages) um = max_pages;
   pl.umax = (int)um;
   pl.tpp = page / kTile;
   const long long groups = (long long)batch * Hkv;
-  const long long tiles = (long long)pl.umax * pl.tpp;
-  long long eps = (tiles * groups + target - 1) / target;  // tiles per split, then pages
-  eps = (eps + pl.tpp - 1) / pl.tpp;
-  if (eps < 1) eps = 1;
-  pl.eps = (int)eps;
-  pl.nsplit = (pl.umax + pl.eps - 1) / pl.eps;
+  long long ns = slots / groups;
+  if (ns > pl.umax) ns = pl.umax;
+  if (ns < 1) ns = 1;
+  pl.nsplit = (int)ns;
+  pl.eps = (pl.umax + pl.nsplit - 1) / pl.nsplit;
   size_t off = 0;
   pl.cnt_off = off;
   off += up256((size_t)batch * Hkv * 4);
@@ -66,46 +70,74 @@ DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, i
 // ---------------------------------------------------------------------------
 // All threads of the CTA call this.  It merges the G heads' selections of
 // (b, g) into per-page head masks in `words` (shared scratch of at least
-// ceil(n/4) words), ranks the selected pages in ascending order with a block
-// scan, stores the entries of rank e0 .. e0 + cap - 1 as page | mask << 24 in
-// `ent` (shared), and returns the union size U.
-__device__ int union_slice(const AttnParams& p, int b, int g, int G, int e0, int cap, uint32_t* words,
-                           uint32_t* ent, int* warp_tot, int* s_cnt) {
-  const int tid = threadIdx.x;
+// ceil(max_pages / 4) words) and ranks the selected pages in ascending order
+// with a block scan.  The union of U pages is cut into nsplit equal slices of
+// ceil(U / nsplit) entries; the entries of slice `split` are stored as
+// page | mask << 24 in `ent` (shared).  Every load of the selections is issued
+// before the first barrier, so their latencies overlap.
+struct UnionSlice {
+  int U;       // union size of (b, g)
+  int e0;      // first union entry of this split
+  int cnt;     // entries in this split (0: no work)
+  int active;  // splits of (b, g) with work
+};
+constexpr int kUnionLoads = 8;  // selection entries a thread loads before the first barrier
+
+__device__ UnionSlice union_slice(const AttnParams& p, int b, int g, int G, int split, uint32_t* words,
+                                  uint32_t* ent, int* warp_tot, int* s_cnt) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
   const int row_len = p.top_k + 2;
   const size_t row0 = (size_t)b * p.Hq + (size_t)g * G;
+  const int total = G * row_len;
+  const int32_t* selg = p.sel + row0 * row_len;  // the G rows are contiguous
   const int L = p.seq_len[b];
-  const int n = max(0, min((L + p.page - 1) / p.page, p.max_pages));
-  const int nw = (n + 3) / 4;
   if (tid < G) s_cnt[tid] = min(p.sel_cnt[row0 + tid], row_len);
-  for (int i = tid; i < nw; i += blockDim.x) words[i] = 0u;
+  int v[kUnionLoads];
+#pragma unroll
+  for (int j = 0; j < kUnionLoads; ++j) {
+    const int i = tid + j * nthr;
+    v[j] = (i < total) ? selg[i] : -1;
+  }
+  for (int i = tid; i < (p.max_pages + 3) / 4; i += nthr) words[i] = 0u;
   __syncthreads();
-  for (int i = tid; i < G * row_len; i += blockDim.x) {
+  const int n = max(0, min((L + p.page - 1) / p.page, p.max_pages));
+  auto mark = [&](int i, int pg) {
     const int hi = i / row_len;
-    if (i - hi * row_len >= s_cnt[hi]) continue;
-    const int pg = p.sel[row0 * row_len + i];
+    if (i - hi * row_len >= s_cnt[hi]) return;
     if (pg < 0 || pg >= n) {
       set_err(p.err, BASISKV_DEVERR_SELECTION);
-      continue;
+      return;
     }
     atomicOr(&words[pg >> 2], (1u << hi) << ((pg & 3) * 8));
+  };
+#pragma unroll
+  for (int j = 0; j < kUnionLoads; ++j) {
+    const int i = tid + j * nthr;
+    if (i < total) mark(i, v[j]);
   }
+  for (int i = tid + kUnionLoads * nthr; i < total; i += nthr) mark(i, selg[i]);
   __syncthreads();
-  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int per = (n + nthr - 1) / nthr;
   const int lo = tid * per, hi = min(n, lo + per);
   int c = 0;
   for (int pg = lo; pg < hi; ++pg) c += ((words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu) ? 1 : 0;
   int tot;
   int pos = block_exclusive_scan(c, warp_tot, tot);
-  for (int pg = lo; pg < hi && pos < e0 + cap; ++pg) {
+  UnionSlice sl;
+  sl.U = tot;
+  const int eps = (tot + p.nsplit - 1) / p.nsplit;
+  sl.e0 = split * eps;
+  sl.cnt = max(0, min(tot, sl.e0 + eps) - sl.e0);
+  sl.active = eps > 0 ? (tot + eps - 1) / eps : 0;
+  for (int pg = lo; pg < hi && pos < sl.e0 + sl.cnt; ++pg) {
     const uint32_t m = (words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu;
     if (m) {
-      if (pos >= e0) ent[pos - e0] = (uint32_t)pg | (m << 24);
+      if (pos >= sl.e0) ent[pos - sl.e0] = (uint32_t)pg | (m << 24);
       ++pos;
     }
   }
   __syncthreads();
-  return tot;
+  return sl;
 }
 
 // Offset of the split's entry list in dynamic shared memory: after the ring
@@ -176,27 +208,51 @@ __device__ __forceinline__ void load_pair(const T* row, int dim, float& a, float
 // spread over `nw` warps starting at warp index `wi`.
 __device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, int g, int G, int r,
                                                    int nsplit_active, int wi, int nw, int lane) {
+  constexpr int kDimIt = 4;  // r <= 128: dims lane + 32 k
+  constexpr int kBatch = 8;  // splits whose values are loaded together
+  const int stride = r + 2;
   for (int hi = wi; hi < G; hi += nw) {
     const int h = g * G + hi;
-    const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * (r + 2);
+    const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * stride;
     float M = -INFINITY;
-    for (int s = lane; s < nsplit_active; s += 32) M = fmaxf(M, __ldcg(base + (size_t)s * (r + 2)));
+    for (int s = lane; s < nsplit_active; s += 32) M = fmaxf(M, __ldcg(base + (size_t)s * stride));
     M = warp_max(M);
     float Ls = 0.f;
-    for (int s = lane; s < nsplit_active; s += 32) {
-      const float ms = __ldcg(base + (size_t)s * (r + 2));
-      if (ms != -INFINITY) Ls += __ldcg(base + (size_t)s * (r + 2) + 1) * exp2f(ms - M);
+    float acc[kDimIt] = {0.f, 0.f, 0.f, 0.f};
+    for (int c0 = 0; c0 < nsplit_active; c0 += 32) {
+      // lane s: the weight of split c0 + s
+      const int sl = c0 + lane;
+      float wl = 0.f;
+      if (sl < nsplit_active) {
+        const float ms = __ldcg(base + (size_t)sl * stride);
+        if (ms != -INFINITY) {
+          wl = exp2f(ms - M);
+          Ls += __ldcg(base + (size_t)sl * stride + 1) * wl;
+        }
+      }
+      const int cn = min(32, nsplit_active - c0);
+      for (int j0 = 0; j0 < cn; j0 += kBatch) {
+        float x[kBatch][kDimIt];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j)
+#pragma unroll
+          for (int k = 0; k < kDimIt; ++k) {
+            const int dim = lane + 32 * k;
+            x[j][k] = (j0 + j < cn && dim < r) ? __ldcg(base + (size_t)(c0 + j0 + j) * stride + 2 + dim) : 0.f;
+          }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const float wt = __shfl_sync(kFull, wl, (j0 + j) & 31);
+#pragma unroll
+          for (int k = 0; k < kDimIt; ++k) acc[k] = fmaf(x[j][k], wt, acc[k]);
+        }
+      }
     }
     Ls = warp_sum(Ls);
-    for (int dim = lane; dim < r; dim += 32) {
-      float a = 0.f;
-      if (M != -INFINITY)
-        for (int s = 0; s < nsplit_active; ++s) {
-          const float* ps = base + (size_t)s * (r + 2);
-          const float ms = __ldcg(ps);
-          if (ms != -INFINITY) a += __ldcg(ps + 2 + dim) * exp2f(ms - M);
-        }
-      p.o_lat[((size_t)b * p.Hq + h) * r + dim] = (Ls > 0.f) ? a / Ls : 0.f;
+#pragma unroll
+    for (int k = 0; k < kDimIt; ++k) {
+      const int dim = lane + 32 * k;
+      if (dim < r) p.o_lat[((size_t)b * p.Hq + h) * r + dim] = (Ls > 0.f) ? acc[k] / Ls : 0.f;
     }
   }
 }
@@ -211,7 +267,6 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.r;
   const size_t bg = (size_t)b * p.Hkv + g;
-  const int e0 = split * p.eps;
   const uint32_t k_bytes = kTile * D * sizeof(T);
   const uint32_t c_bytes = kTile * r * sizeof(T);
   const uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
@@ -219,16 +274,16 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   uint32_t* ent = reinterpret_cast<uint32_t*>(smem + attn_ent_offset(kStages * stage_bytes + 2 * kStages * 8, p.max_pages));
   __shared__ int warp_tot[32];
   __shared__ int s_cnt[8];
-  const int U = union_slice(p, b, g, G, e0, p.eps, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
-  const int nsplit_active = (U + p.eps - 1) / p.eps;
-  if (e0 >= U) {
+  const UnionSlice sl = union_slice(p, b, g, G, split, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
+  const int U = sl.U, nsplit_active = sl.active;
+  if (sl.cnt == 0) {
     // no work in this split; split 0 of an empty group still defines its output
     if (split == 0 && U == 0)
       for (int i = threadIdx.x; i < G * r; i += blockDim.x)
         p.o_lat[((size_t)b * p.Hq + (size_t)g * G) * r + i] = 0.f;
     return;
   }
-  const int nent = min(U, e0 + p.eps) - e0;
+  const int nent = sl.cnt;
   const int ntiles = nent * p.tpp;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * stage_bytes);
   uint64_t* empty = full + kStages;
@@ -251,7 +306,7 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
     const T* kbase = static_cast<const T*>(p.k_raw);
     const T* cbase = static_cast<const T*>(p.c_lat);
     for (int cb = 0; cb < nent && ok; cb += 32) {
-      // lane e holds union entry e0 + cb + e
+      // lane e holds entry cb + e of this split
       uint32_t my_mask = 0;
       int my_phys = -1, my_valid = 0;
       if (cb + lane < nent) {
@@ -401,7 +456,6 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
 // ---------------------------------------------------------------------------
 constexpr int kMmaWarps = 4;       // warps per CTA; each streams and consumes its own tiles
 constexpr int kMmaWarpStages = 3;  // ring slots per warp
-constexpr int kMmaTargetCtas = 444;  // one wave at 3 CTAs per SM
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -437,7 +491,6 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   uint32_t* meta = meta_all[w];
   const size_t bg = (size_t)b * p.Hkv + g;
-  const int e0 = split * p.eps;
   constexpr uint32_t k_bytes = kTile * D * 2;
   constexpr uint32_t c_bytes = kTile * R * 2;
   constexpr uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
@@ -446,15 +499,15 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
   uint32_t* ent = reinterpret_cast<uint32_t*>(smem + attn_ent_offset(ring_bytes, p.max_pages));
   __shared__ int warp_tot[32];
   __shared__ int s_cnt[8];
-  const int U = union_slice(p, b, g, G, e0, p.eps, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
-  const int nsplit_active = (U + p.eps - 1) / p.eps;
-  if (e0 >= U) {
+  const UnionSlice sl = union_slice(p, b, g, G, split, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
+  const int U = sl.U, nsplit_active = sl.active;
+  if (sl.cnt == 0) {
     if (split == 0 && U == 0)
       for (int i = threadIdx.x; i < G * R; i += blockDim.x)
         p.o_lat[((size_t)b * p.Hq + (size_t)g * G) * R + i] = 0.f;
     return;
   }
-  const int nent = min(U, e0 + p.eps) - e0;
+  const int nent = sl.cnt;
   const int ntiles = nent * p.tpp;
 
   unsigned char* ring = smem + (size_t)w * SW * stage_bytes;

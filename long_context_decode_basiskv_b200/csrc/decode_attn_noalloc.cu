@@ -64,8 +64,11 @@ extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
   if (cache->max_pages <= 0) return BASISKV_ERR_INVALID_ARG;
 
   // the same scratch basiskv_decode_attn takes from its workspace
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const DecodePlan plan = decode_plan(cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v, cfg->top_k,
-                                      batch, cache->max_pages, cfg->dtype == BASISKV_BF16, cfg->head_dim);
+                                      batch, cache->max_pages, cfg->dtype == BASISKV_BF16, cfg->head_dim,
+                                      sms > 0 ? sms : 148);
   if (plan.bytes > kNoAllocScratchBytes) {
     fprintf(stderr,
             "basiskv_decode_attn_noalloc: this shape needs %zu bytes of scratch, more than the "

@@ -61,7 +61,8 @@ struct DecodePlan {
   int nsplit;  // splits per (sequence, KV head)
   size_t cnt_off, part_off, bytes;
 };
-DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d);
+DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d,
+                       int num_sms);
 
 struct DecodeArgs {
   const void* q;
