@@ -38,9 +38,13 @@ constexpr int kMmaCtasPerSm = 3;    // ... and of the tensor-core one (registers
 // ---------------------------------------------------------------------------
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Every (sequence, KV head) group gets the same number of splits, as many as
-// one resident wave of the kernel holds (at least one); each split takes an
-// equal share of its group's union at run time, at most eps pages.
+// The splits fill one resident wave of the kernel exactly: with q = slots /
+// groups and m = slots % groups, the last m groups get q + 1 splits and the
+// others q (at least one each), so every SM holds the same number of CTAs and
+// about the same number of tiles (the memory system gives every SM a similar
+// share of the bandwidth, so an SM with more work would finish last).  Each
+// split takes an equal share of its group's union at run time.  The first
+// groups' unused CTAs (split q) exit at once and free their slots.
 DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d,
                        int num_sms) {
   DecodePlan pl{};
@@ -51,11 +55,19 @@ DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, i
   pl.umax = (int)um;
   pl.tpp = page / kTile;
   const long long groups = (long long)batch * Hkv;
-  long long ns = slots / groups;
-  if (ns > pl.umax) ns = pl.umax;
-  if (ns < 1) ns = 1;
-  pl.nsplit = (int)ns;
-  pl.eps = (pl.umax + pl.nsplit - 1) / pl.nsplit;
+  long long q = slots / groups, m = slots % groups;
+  if (q >= pl.umax) {
+    q = pl.umax;
+    m = 0;
+  }
+  if (q < 1) {
+    q = 1;
+    m = 0;
+  }
+  pl.nsplit_lo = (int)q;
+  pl.nsplit = (int)(m > 0 ? q + 1 : q);
+  pl.rich_from = (int)(groups - m);
+  pl.eps = (pl.umax + pl.nsplit_lo - 1) / pl.nsplit_lo;
   size_t off = 0;
   pl.cnt_off = off;
   off += up256((size_t)batch * Hkv * 4);
@@ -125,9 +137,10 @@ __device__ UnionSlice union_slice(const AttnParams& p, int b, int g, int G, int 
   int pos = block_exclusive_scan(c, warp_tot, tot);
   UnionSlice sl;
   sl.U = tot;
-  const int eps = (tot + p.nsplit - 1) / p.nsplit;
+  const int ns = ((int)(b * p.Hkv + g) >= p.rich_from) ? p.nsplit : p.nsplit_lo;  // splits of this group
+  const int eps = (tot + ns - 1) / ns;
   sl.e0 = split * eps;
-  sl.cnt = max(0, min(tot, sl.e0 + eps) - sl.e0);
+  sl.cnt = (split < ns) ? max(0, min(tot, sl.e0 + eps) - sl.e0) : 0;
   sl.active = eps > 0 ? (tot + eps - 1) / eps : 0;
   for (int pg = lo; pg < hi && pos < sl.e0 + sl.cnt; ++pg) {
     const uint32_t m = (words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu;
@@ -146,6 +159,12 @@ __host__ __device__ __forceinline__ size_t attn_ent_offset(size_t ring_bytes, in
   const size_t masks = ((size_t)max_pages + 15) & ~(size_t)15;
   return ((ring_bytes > masks ? ring_bytes : masks) + 15) & ~(size_t)15;
 }
+
+// The out-projection is launched as a programmatic dependent of this kernel:
+// letting it launch at once lets its CTAs take SMs as soon as attention CTAs
+// retire and start streaming their weights; it waits for this grid to finish
+// before it reads o_lat.
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // After writing its split results, a CTA counts itself on the group's counter;
 // the last one of the group merges.  The merging CTA puts the counter back to
@@ -260,6 +279,7 @@ __device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, i
 template <typename T, int D, int G, int CU>
 __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   constexpr int DPL = D / 32;
+  allow_dependents();
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint32_t meta[kStages];  // head mask | valid tokens << 8 of the tile in each stage
   __shared__ int s_last;
@@ -482,6 +502,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int D, int G, int NT>
 __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams p) {
   constexpr int KS = D / 16;
+  allow_dependents();
   constexpr int SW = kMmaWarpStages;
   constexpr int R = NT * 8;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -809,7 +830,7 @@ cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* 
   float* part = reinterpret_cast<float*>(base + pl.part_off);
   AttnParams ap{a.q, a.k_raw, a.c_lat, a.block_table, a.seq_len, a.sel, a.sel_cnt, cnt, part, a.o_lat, a.err,
                 a.Hq, a.Hkv, a.page, a.r, a.max_pages, a.num_phys, a.top_k, pl.umax, pl.tpp, pl.eps, pl.nsplit,
-                (float)(1.4426950408889634 / sqrt((double)a.d))};
+                pl.nsplit_lo, pl.rich_from, (float)(1.4426950408889634 / sqrt((double)a.d))};
   cudaError_t e;
   const int G = a.Hq / a.Hkv;
   (void)e;

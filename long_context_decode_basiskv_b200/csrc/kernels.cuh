@@ -48,7 +48,7 @@ struct AttnParams {
   float* part;   // [B][Hq][nsplit][r + 2]
   float* o_lat;  // [B][Hq][r]
   int32_t* err;
-  int Hq, Hkv, page, r, max_pages, num_phys, top_k, umax, tpp, eps, nsplit;
+  int Hq, Hkv, page, r, max_pages, num_phys, top_k, umax, tpp, eps, nsplit, nsplit_lo, rich_from;
   float qscale;  // log2(e) / sqrt(d)
 };
 
@@ -57,8 +57,10 @@ struct AttnParams {
 struct DecodePlan {
   int umax;    // max union pages per (sequence, KV head)
   int tpp;     // 16-token tiles per page
-  int eps;     // union pages per split
-  int nsplit;  // splits per (sequence, KV head)
+  int eps;        // union pages per split, at most
+  int nsplit;     // splits of the groups with the most (grid x extent; partial slots per head)
+  int nsplit_lo;  // splits of groups b * Hkv + g < rich_from (nsplit or nsplit - 1)
+  int rich_from;
   size_t cnt_off, part_off, bytes;
 };
 DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d,

@@ -19,10 +19,15 @@
 // were committed; warps 1-4 prefetch the matching slices of o with cp.async,
 // write them as swizzled bf16 hi/lo tiles into a matching ring and, at the
 // end, read the accumulator out of TMEM.
-// The K dimension is split over the CTAs of a thread-block cluster; their
-// partial tiles are summed through distributed shared memory in a fixed
-// order (deterministic), each CTA writing a slice of the output rows.
+// The K dimension is split over the CTAs of a thread-block cluster.  Each CTA
+// stores its partial rows straight into the shared memory of the CTA that
+// owns them (distributed shared memory stores); after one cluster barrier
+// every CTA sums its slice of rows in rank order (deterministic) and writes y.
 // HBM-bound: Gt is read once (16.8 MB for the 32K Llama-3-8B shape).
+//
+// The kernel is launched as a programmatic dependent of the attention kernel
+// that produces o: the Gt stream starts as soon as SMs free up, and only the
+// threads that read o wait (griddepcontrol.wait) for the producer to finish.
 #include <stdio.h>
 
 #include "kernels.cuh"
@@ -82,13 +87,18 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float ld_dsmem_f32(const float* local, uint32_t rank) {
+// 16-byte store into the shared memory of CTA `rank` of the cluster, at the
+// address that `local` has in this CTA
+__device__ __forceinline__ void st_dsmem_v4(const float* local, uint32_t rank, float4 v) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
 }
+
+// wait until the grids this one depends on have completed and their writes are visible
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // K-major operand tile in shared memory, 128-byte swizzle: rows of 128 bytes,
 // 8-row groups 1024 bytes apart.  Start address advanced by 32 bytes per
@@ -111,7 +121,8 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// ring depth per batch tile width (shared memory: A 16 KB, B 2*NB*128 B, o staging NB*256 B per stage)
+// ring depth per batch tile width (shared memory: A 16 KB, B 2*NB*128 B, o staging NB*256 B per stage;
+// plus the 128 x NB fp32 receive buffer of the cluster reduction)
 template <int NB>
 struct TcStages {
   static constexpr int S = NB <= 16 ? 8 : NB <= 32 ? 6 : 4;
@@ -130,12 +141,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   unsigned char* sA = smem;
   unsigned char* sB = smem + S * kTcABytes;
   unsigned char* sO = sB + S * 2 * kBBytes;
-  uint64_t* afull = reinterpret_cast<uint64_t*>(sO + S * kStageF32);
+  float* recv = reinterpret_cast<float*>(sO + S * kStageF32);  // [ksplit][rows][NB]: partial rows from every rank
+  uint64_t* afull = reinterpret_cast<uint64_t*>(recv + kTcM * NB);
   uint64_t* bfull = afull + S;
   uint64_t* empty = bfull + S;
   uint64_t* done = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  float* red = reinterpret_cast<float*>(smem);  // [128][NB], reuses the A ring after the last MMA
   __shared__ int s_fail;  // a bounded wait gave up: the outputs of this cluster become NaN
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,6 +177,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // this CTA has started; the matching wait comes before the first store into a peer's shared memory
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
@@ -216,6 +229,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // stage; they are prefetched S stages ahead with cp.async into fp32 staging,
     // then split into bf16 hi / lo and written in the operand's swizzled layout
     const int t = threadIdx.x - 32;
+    grid_dep_wait();  // o is written by the kernel this one follows
     auto issue = [&](int i) {
       unsigned char* stg = sO + (i % S) * kStageF32;
 #pragma unroll
@@ -277,36 +291,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     set_err(p.err, BASISKV_DEVERR_TIMEOUT);
   }
   tc_fence_after();
-  __syncthreads();  // every TMA landed and every MMA done: the A ring is free for `red`
-  fence_proxy_async_smem();
+  __syncthreads();
+  // accumulator row m goes to the CTA that owns it: rank m / rows, slot [rank][m % rows]
+  const int rows = kTcM / p.ksplit;
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA of the cluster is running
   if (warp >= 1) {
     const int q = warp & 3;
     const int m = q * 32 + lane;
+    const uint32_t owner = (uint32_t)(m / rows);
+    float* slot = recv + ((size_t)rank * rows + (m % rows)) * NB;
 #pragma unroll
     for (int cc = 0; cc < NB; cc += 16) {
       float v[16];
       tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cc, v);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) red[m * NB + cc + j] = (nst > 0) ? v[j] : 0.f;
+      for (int j = 0; j < 16; j += 4) {
+        const float4 x = (nst > 0) ? make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        st_dsmem_v4(slot + cc + j, owner, x);
+      }
     }
   }
   tc_fence_before();
-  cluster_sync();
-
-  // each CTA of the cluster sums its slice of rows over the cluster, in rank order
-  const int rows = kTcM / p.ksplit;
-  const int r0 = (int)rank * rows;
-  for (int idx = threadIdx.x; idx < rows * NB; idx += blockDim.x) {
-    const int n = idx / rows, m = r0 + idx % rows;
-    float acc = 0.f;
-    for (int q = 0; q < p.ksplit; ++q) acc += ld_dsmem_f32(red + m * NB + n, (uint32_t)q);
-    if (s_fail) acc = __int_as_float(0x7fc00000);  // NaN marks a result that cannot be trusted
-    if (b0 + n < p.batch) p.y[(size_t)(b0 + n) * p.hidden + c0 + m] = acc;
-  }
-  cluster_sync();  // no CTA leaves while its shared memory may still be read
+  cluster_sync();  // every partial row has landed in its owner's receive buffer
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
+  }
+  // this CTA's rows r0 .. r0 + rows - 1, summed over the ranks in order
+  const int r0 = (int)rank * rows;
+  for (int idx = threadIdx.x; idx < rows * NB; idx += blockDim.x) {
+    const int n = idx / rows, mm = idx % rows;
+    float acc = 0.f;
+    for (int q = 0; q < p.ksplit; ++q) acc += recv[((size_t)q * rows + mm) * NB + n];
+    if (s_fail) acc = __int_as_float(0x7fc00000);  // NaN marks a result that cannot be trusted
+    if (b0 + n < p.batch) p.y[(size_t)(b0 + n) * p.hidden + c0 + r0 + mm] = acc;
   }
 }
 
@@ -318,7 +336,8 @@ bool gt_blocked(int K, int hidden) { return K % kTcK == 0 && hidden % kTcM == 0;
 template <int NB>
 static size_t tc_smem_bytes() {
   constexpr int S = TcStages<NB>::S;
-  return 1024 + (size_t)S * kTcABytes + (size_t)S * 2 * NB * kTcK * 2 + (size_t)S * NB * kTcK * 4 + (3 * S + 1) * 8 + 16;
+  return 1024 + (size_t)S * kTcABytes + (size_t)S * 2 * NB * kTcK * 2 + (size_t)S * NB * kTcK * 4 +
+         (size_t)kTcM * NB * 4 + (3 * S + 1) * 8 + 16;
 }
 
 template <int NB>
@@ -338,13 +357,15 @@ static cudaError_t launch_tc_nb(OutProjTcParams p, int num_sms, cudaStream_t st)
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start before the o producer ends
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, out_proj_tc_kernel<NB>, p);
 }
 
