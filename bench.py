@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--workload", default="llama3_8b_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--oracle-seqs", type=int, default=2, help="sequences in the CPU-baseline sample")
+    ap.add_argument("--oracle-repeats", type=int, default=100,
+                    help="decode steps per sampled sequence in the CPU baseline (about 10 s in total)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -371,7 +373,7 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, desc = oracle_sample(case, args.oracle_seqs)
+        times, desc = oracle_sample(case, args.oracle_seqs, args.oracle_repeats)
         cpu = {"value": round(len(times) / sum(times), 3), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": desc, "seconds": round(sum(times), 3)}
 

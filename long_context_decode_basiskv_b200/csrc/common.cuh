@@ -203,6 +203,17 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 
+// -------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running; it must execute grid_dep_wait() before it reads anything that
+// kernel wrote.  A kernel calls allow_dependents() to let its dependent launch
+// early.  Both instructions are no-ops when there is no such dependency.
+// -------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+
 // Raise a kernel's dynamic shared memory limit once per (device, kernel), so
 // that later calls (including calls made while a stream is being captured
 // into a CUDA graph) launch without touching function attributes.

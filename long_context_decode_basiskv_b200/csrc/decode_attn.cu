@@ -160,12 +160,6 @@ __host__ __device__ __forceinline__ size_t attn_ent_offset(size_t ring_bytes, in
   return ((ring_bytes > masks ? ring_bytes : masks) + 15) & ~(size_t)15;
 }
 
-// The out-projection is launched as a programmatic dependent of this kernel:
-// letting it launch at once lets its CTAs take SMs as soon as attention CTAs
-// retire and start streaming their weights; it waits for this grid to finish
-// before it reads o_lat.
-__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // After writing its split results, a CTA counts itself on the group's counter;
 // the last one of the group merges.  The merging CTA puts the counter back to
 // zero, so counters are zero between calls (the workspace is zero-filled once).
@@ -279,7 +273,7 @@ __device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, i
 template <typename T, int D, int G, int CU>
 __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   constexpr int DPL = D / 32;
-  allow_dependents();
+  allow_dependents();  // the out-projection may launch and start streaming its weights
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint32_t meta[kStages];  // head mask | valid tokens << 8 of the tile in each stage
   __shared__ int s_last;
@@ -502,7 +496,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 template <int D, int G, int NT>
 __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams p) {
   constexpr int KS = D / 16;
-  allow_dependents();
+  allow_dependents();  // the out-projection may launch and start streaming its weights
   constexpr int SW = kMmaWarpStages;
   constexpr int R = NT * 8;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -765,8 +759,7 @@ static cudaError_t launch_attn_t(const AttnParams& p, int batch, cudaStream_t st
   const size_t smem = attn_smem_bytes(D, p.r, sizeof(T), p.max_pages, p.eps);
   cudaError_t e = ensure_smem((const void*)attn_kernel<T, D, G, CU>, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nsplit, p.Hkv, batch);
-  attn_kernel<T, D, G, CU><<<grid, 32 * (G + 1), smem, st>>>(p);
+  attn_kernel<T, D, G, CU><<<dim3(p.nsplit, p.Hkv, batch), 32 * (G + 1), smem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -97,8 +97,6 @@ __device__ __forceinline__ void st_dsmem_v4(const float* local, uint32_t rank, f
                : "memory");
 }
 
-// wait until the grids this one depends on have completed and their writes are visible
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // K-major operand tile in shared memory, 128-byte swizzle: rows of 128 bytes,
 // 8-row groups 1024 bytes apart.  Start address advanced by 32 bytes per
