@@ -115,7 +115,13 @@ basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* ca
   AppendParams p{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
                  cache->summary, cache->block_table, cache->seq_len, err_flag,
                  batch, n_new, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
-                 cfg->page_size, cache->max_pages, cache->num_phys_pages};
+                 cfg->page_size, cache->max_pages, cache->num_phys_pages, nullptr, 0};
+  // the decode step's out-projection reads the whole fused factor: start bringing it into L2 now
+  const size_t gt_bytes = (size_t)cfg->hidden * cfg->num_q_heads * cfg->rank_v * esize(cfg);
+  if (n_new == 1 && f->Gt && aligned16(f->Gt) && gt_bytes % 16 == 0) {
+    p.warm = f->Gt;
+    p.warm_bytes = gt_bytes;
+  }
   return cuda_status(launch_append(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
 }
 

@@ -565,6 +565,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
       }
     }
   };
+  const uint64_t stream_pol = l2_evict_first();
   // issue tile i of this warp into slot i % SW (lane 0); all lanes take part in the shuffles
   auto issue = [&](int i) {
     const int j = i & 31;
@@ -580,8 +581,8 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
         const int pidx = ph / p.tpp, sub = ph - pidx * p.tpp;
         const size_t row0 = ((size_t)pidx * p.Hkv + g) * p.page + (size_t)sub * kTile;
         mbar_arrive_expect_tx(bar, k_bytes + c_bytes);
-        bulk_g2s(st, kbase + row0 * D, k_bytes, bar);
-        bulk_g2s(st + k_bytes, cbase + row0 * R, c_bytes, bar);
+        bulk_g2s_hint(st, kbase + row0 * D, k_bytes, bar, stream_pol);  // read once: evict first
+        bulk_g2s_hint(st + k_bytes, cbase + row0 * R, c_bytes, bar, stream_pol);
       } else {
         mbar_arrive_expect_tx(bar, 0);
       }

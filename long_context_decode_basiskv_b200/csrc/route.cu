@@ -84,10 +84,10 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
       if (ph >= 0) {
         const float* rowp = p.summary + ((size_t)ph * p.Hkv + g) * D + lane * DPL;
         if constexpr (DPL == 4) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(rowp));
+          const float4 v = __ldcs(reinterpret_cast<const float4*>(rowp));  // read once: evict first
           sv[i][0] = v.x; sv[i][1] = v.y; sv[i][2] = v.z; sv[i][3] = v.w;
         } else {
-          const float2 v = __ldg(reinterpret_cast<const float2*>(rowp));
+          const float2 v = __ldcs(reinterpret_cast<const float2*>(rowp));
           sv[i][0] = v.x; sv[i][1] = v.y;
         }
       } else {
