@@ -172,6 +172,8 @@ basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors
   (void)ws;
   (void)ws_bytes;
   const int K = cfg->num_q_heads * cfg->rank_v;
+  if (cfg->dtype == BASISKV_BF16 && out_proj_mma_fits(batch, K, cfg->hidden))
+    return cuda_status(launch_out_proj_mma(o_lat, f->Gt, y, batch, K, cfg->hidden, (cudaStream_t)stream));
   if (cfg->dtype == BASISKV_BF16 && gt_blocked(K, cfg->hidden))
     return cuda_status(launch_out_proj_tc(o_lat, f->Gt, y, nullptr, batch, K, cfg->hidden, num_sms(),
                                           (cudaStream_t)stream));

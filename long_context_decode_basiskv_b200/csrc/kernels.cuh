@@ -94,6 +94,10 @@ cudaError_t launch_out_proj_gemv(const OutProjParams& p, bool bf16, cudaStream_t
 // bf16 shapes with K % 64 == 0 and hidden % 128 == 0 keep Gt in the blocked
 // tensor-core layout (see out_proj_tc.cu); every other shape uses [hidden][K].
 bool gt_blocked(int K, int hidden);
+// small batches (<= 8) with the pre-tiled Gt: mma.sync kernel without cluster or tensor memory
+bool out_proj_mma_fits(int batch, int K, int hidden);
+cudaError_t launch_out_proj_mma(const float* o, const void* Gt, float* y, int batch, int K, int hidden,
+                                cudaStream_t st);
 cudaError_t launch_out_proj_tc(const float* o, const void* Gt, float* y, int32_t* err, int batch, int K, int hidden,
                                int num_sms, cudaStream_t st);
 

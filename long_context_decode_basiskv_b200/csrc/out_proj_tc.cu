@@ -126,6 +126,16 @@ struct TcStages {
   static constexpr int S = NB <= 16 ? 8 : NB <= 32 ? 6 : 4;
 };
 
+// The MMAs of one accumulator execute one after another; spreading the K-steps
+// over kTcAcc accumulators (one per K = 16 slice of a stage and per hi / lo
+// half) keeps the tensor core busy with independent chains.  The epilogue sums
+// the accumulators.
+constexpr int kTcAcc = 8;
+template <int NB>
+struct TcCols {  // TMEM columns: kTcAcc accumulators of NB fp32 columns, a power of two >= 32
+  static constexpr uint32_t n = kTcAcc * NB <= 128 ? 128u : kTcAcc * NB <= 256 ? 256u : 512u;
+};
+
 template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     out_proj_tc_kernel(OutProjTcParams p) {
@@ -133,7 +143,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   constexpr uint32_t kBBytes = NB * kTcK * 2;       // one of hi / lo per stage
   constexpr uint32_t kStageF32 = NB * kTcK * 4;     // fp32 staging of o per stage
   constexpr int kChunks = NB * 8 / 128;            // 8-float chunks per producer thread per stage
-  constexpr uint32_t kCols = NB <= 32 ? 32 : 64;
+  constexpr uint32_t kCols = TcCols<NB>::n;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* sA = smem;
@@ -203,8 +213,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int j = 0; j < kTcK / 16; ++j) {
           const uint64_t step = (uint64_t)(j * 32) >> 4;  // 32 bytes per K = 16 slice
-          tc_mma(tmem, ad + step, bh + step, idesc, (i > 0 || j > 0) ? 1u : 0u);
-          tc_mma(tmem, ad + step, bl + step, idesc, 1u);
+          const uint32_t acc_h = tmem + (uint32_t)(2 * j) * NB, acc_l = acc_h + NB;
+          tc_mma(acc_h, ad + step, bh + step, idesc, i > 0 ? 1u : 0u);
+          tc_mma(acc_l, ad + step, bl + step, idesc, i > 0 ? 1u : 0u);
         }
         tc_commit(&empty[s]);
         // refill the stage of the previous iteration (its MMAs have had a whole iteration to finish)
@@ -302,6 +313,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int cc = 0; cc < NB; cc += 16) {
       float v[16];
       tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)cc, v);
+#pragma unroll
+      for (int a = 1; a < kTcAcc; ++a) {
+        float u[16];
+        tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NB + cc), u);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] += u[j];
+      }
 #pragma unroll
       for (int j = 0; j < 16; j += 4) {
         const float4 x = (nst > 0) ? make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
