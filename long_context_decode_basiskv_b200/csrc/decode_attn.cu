@@ -274,6 +274,7 @@ template <typename T, int D, int G, int CU>
 __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   constexpr int DPL = D / 32;
   allow_dependents();  // the out-projection may launch and start streaming its weights
+  grid_dep_wait();     // the selection is complete (this kernel may launch before it ends)
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint32_t meta[kStages];  // head mask | valid tokens << 8 of the tile in each stage
   __shared__ int s_last;
@@ -497,6 +498,7 @@ template <int D, int G, int NT>
 __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams p) {
   constexpr int KS = D / 16;
   allow_dependents();  // the out-projection may launch and start streaming its weights
+  grid_dep_wait();     // the selection is complete (this kernel may launch before it ends)
   constexpr int SW = kMmaWarpStages;
   constexpr int R = NT * 8;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -750,6 +752,25 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
 // ---------------------------------------------------------------------------
 // launch
 // ---------------------------------------------------------------------------
+// The attention kernels launch as programmatic dependents of the selection
+// kernel before them on the stream: their CTAs may start while it finishes and
+// wait (grid_dep_wait) before reading anything.
+template <typename K>
+static cudaError_t launch_dependent_of_route(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                            const AttnParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 size_t attn_smem_bytes(int d, int r, int esize, int max_pages, int eps) {
   const size_t stage = ((size_t)kTile * (d + r) * esize + 127) & ~(size_t)127;
   return attn_ent_offset((size_t)kStages * stage + 2 * kStages * 8, max_pages) + (size_t)eps * 4;
@@ -760,8 +781,8 @@ static cudaError_t launch_attn_t(const AttnParams& p, int batch, cudaStream_t st
   const size_t smem = attn_smem_bytes(D, p.r, sizeof(T), p.max_pages, p.eps);
   cudaError_t e = ensure_smem((const void*)attn_kernel<T, D, G, CU>, smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<T, D, G, CU><<<dim3(p.nsplit, p.Hkv, batch), 32 * (G + 1), smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_dependent_of_route(attn_kernel<T, D, G, CU>, dim3(p.nsplit, p.Hkv, batch), dim3(32 * (G + 1)),
+                                   smem, st, p);
 }
 
 template <typename T, int D, int G>
@@ -787,8 +808,8 @@ static cudaError_t launch_mma_t(const AttnParams& p, int batch, cudaStream_t st)
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem((const void*)attn_mma_kernel<D, G, NT>, smem);
   if (e != cudaSuccess) return e;
-  attn_mma_kernel<D, G, NT><<<dim3(p.nsplit, p.Hkv, batch), 32 * kMmaWarps, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_dependent_of_route(attn_mma_kernel<D, G, NT>, dim3(p.nsplit, p.Hkv, batch), dim3(32 * kMmaWarps),
+                                   smem, st, p);
 }
 
 template <int D, int G>

@@ -158,6 +158,7 @@ template <int KPT>
 __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
   __shared__ int red[2 * kSelectWarps];
   __shared__ int warp_tot[32];
+  allow_dependents();  // the attention kernel may launch; it waits for this selection
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int L = p.seq_len[b];
   const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
@@ -291,6 +292,7 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(Route
   __shared__ float cand[kCandCap];
   __shared__ int s_ncand, s_D, s_above, s_rem;
   __shared__ float s_T;
+  allow_dependents();
 
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x;
