@@ -109,7 +109,7 @@ class ClockSampler:
         "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
     }
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.ok = False
         try:
             import pynvml
@@ -353,7 +353,7 @@ def run_ours(args, world, rank, local):
                     eng.q.copy_(hq, non_blocking=True)
                     eng.k_new.copy_(hk, non_blocking=True)
                     eng.v_new.copy_(hv, non_blocking=True)
-                    eng.step()
+                    eng.graph_step()
                     hy.copy_(eng.y, non_blocking=True)
                     if record:
                         b_.record(stream)

@@ -101,6 +101,22 @@ class DecodeEngine:
         self.out_proj(stream)
         return self.y
 
+    def graph_step(self):
+        """step() replayed from a CUDA graph captured on first use (the inputs are
+        read from and the outputs written to the engine's tensors, so a caller
+        refreshes q / k_new / v_new in place between steps)."""
+        if not hasattr(self, "_graph"):
+            side = torch.cuda.Stream(device=self.device)
+            side.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(side):
+                self.step()  # first launches (shared-memory attributes) outside the capture
+            torch.cuda.current_stream(self.device).wait_stream(side)
+            self._graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self._graph, stream=side):
+                self.step()
+        self._graph.replay()
+        return self.y
+
     def kc_swizzled(self) -> bool:
         """bf16 K and C pages are stored with 16-byte chunks XOR-swizzled per row."""
         c = self.cfg

@@ -108,3 +108,21 @@ def test_workspace_too_small_is_rejected():
     with pytest.raises(bk.BasisKVError) as ei:
         bk.route(eng.cfg, eng.cache, eng.q, eng.sel, eng.sel_cnt, small, eng.err)
     assert ei.value.status == bk.ERR_WORKSPACE
+
+
+def test_graph_step_matches_step():
+    """The engine's CUDA-graph step gives exactly the eager step's outputs, also when replayed."""
+    wl = shrink(WORKLOADS["llama3_8b_32k"], batch=3, context=16 * 300 + 7, top_k=24, name="graph_step")
+    eng = DecodeEngine(make_case(wl, "cuda"))
+    eng.step()
+    torch.cuda.synchronize()
+    ref = (eng.sel.clone(), eng.o_lat.clone(), eng.y.clone())
+    for _ in range(2):
+        eng.y.zero_()
+        eng.o_lat.zero_()
+        eng.graph_step()
+        torch.cuda.synchronize()
+        assert int(eng.err.item()) == 0
+        assert torch.equal(eng.sel, ref[0])
+        assert torch.equal(eng.o_lat, ref[1])
+        assert torch.equal(eng.y, ref[2])
