@@ -335,11 +335,9 @@ def run_ours(args, world, rank, local):
     # end to end through the public API: pinned host inputs -> step -> host output
     e2e = None
     if not args.no_e2e:
-        hq = eng.q.cpu().pin_memory()
-        hk = eng.k_new.cpu().pin_memory()
-        hv = eng.v_new.cpu().pin_memory()
+        hin = eng.input_buffer().cpu().pin_memory()   # q, k_new, v_new of the step, packed
         hy = torch.empty(eng.y.shape, dtype=eng.y.dtype).pin_memory()
-        bi = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+        bi = hin.numel() * hin.element_size()
         bo = hy.numel() * hy.element_size()
 
         def e2e_steps(n, record):
@@ -350,9 +348,7 @@ def run_ours(args, world, rank, local):
                     if record:
                         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                         a.record(stream)
-                    eng.q.copy_(hq, non_blocking=True)
-                    eng.k_new.copy_(hk, non_blocking=True)
-                    eng.v_new.copy_(hv, non_blocking=True)
+                    eng.input_buffer().copy_(hin, non_blocking=True)
                     eng.graph_step()
                     hy.copy_(eng.y, non_blocking=True)
                     if record:

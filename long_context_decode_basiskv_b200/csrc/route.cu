@@ -43,27 +43,28 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
   __shared__ __align__(16) float sq[G * D];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the length, this lane's block-table entry and the query rows are loaded
+  // together (the entry is validated once the length is known)
+  const int pw0 = c * kScoreCtaPages + warp * kScoreWarpPages;
+  const int pl = pw0 + lane;
+  const int raw_phys = (pl < p.max_pages) ? p.block_table[(size_t)b * p.max_pages + pl] : -1;
   const int L = p.seq_len[b];
   int n = (L + p.page - 1) / p.page;
   if (n > p.max_pages) {
     if (c == 0 && tid == 0) set_err(p.err, BASISKV_DEVERR_SEQ_LEN);
     n = p.max_pages;
   }
-  const int pw0 = c * kScoreCtaPages + warp * kScoreWarpPages;
   if (c * kScoreCtaPages >= n) return;  // the whole CTA is past the last page
   const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;
   const T* qb = static_cast<const T*>(p.q) + qrow * D;
   for (int i = tid; i < G * D; i += kScoreThreads) sq[i] = Elem<T>::to_f(qb[i]);
 
   int my_phys = -1;  // -1: not scored, -2: bad block-table entry
-  {
-    const int pl = pw0 + lane;
-    if (pl < n && (p.all_pages || (pl != 0 && pl != n - 1))) {
-      my_phys = p.block_table[(size_t)b * p.max_pages + pl];
-      if (my_phys < 0 || my_phys >= p.num_phys) {
-        set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
-        my_phys = -2;
-      }
+  if (pl < n && (p.all_pages || (pl != 0 && pl != n - 1))) {
+    my_phys = raw_phys;
+    if (my_phys < 0 || my_phys >= p.num_phys) {
+      set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
+      my_phys = -2;
     }
   }
   __syncthreads();  // sq

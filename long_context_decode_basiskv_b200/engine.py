@@ -37,16 +37,32 @@ class DecodeEngine:
                            self.factors.Gt, stream)
         self.err = torch.zeros(1, dtype=torch.int32, device=dev)
         self.ws = bk.alloc_workspace(cfg, B, self.cache.max_pages, device=dev)
-        # step inputs: the last token of every sequence, and the query
-        self.k_new = torch.stack([k[-1] for k in case.keys]).unsqueeze(1).to(dev).contiguous()
-        self.v_new = torch.stack([v[-1] for v in case.values]).unsqueeze(1).to(dev).contiguous()
-        self.q = case.q.to(dev).contiguous()
+        # step inputs: the last token of every sequence, and the query; q, k_new
+        # and v_new are views of one device buffer, so a caller can refresh all
+        # three with one host-to-device copy (input_buffer)
+        k_new = torch.stack([k[-1] for k in case.keys]).unsqueeze(1)
+        v_new = torch.stack([v[-1] for v in case.values]).unsqueeze(1)
+        q = case.q
+        parts = [q, k_new, v_new]
+        sizes = [t.numel() for t in parts]
+        self._inbuf = torch.empty(sum(sizes), dtype=cfg.dtype, device=dev)
+        views, off = [], 0
+        for t, n in zip(parts, sizes):
+            v = self._inbuf[off:off + n].view(t.shape)
+            v.copy_(t.to(dev))
+            views.append(v)
+            off += n
+        self.q, self.k_new, self.v_new = views
         # step outputs
         self.sel = torch.empty((B, cfg.num_q_heads, cfg.top_k + 2), dtype=torch.int32, device=dev)
         self.sel_cnt = torch.empty((B, cfg.num_q_heads), dtype=torch.int32, device=dev)
         self.o_lat = torch.empty((B, cfg.num_q_heads, cfg.rank_v), dtype=torch.float32, device=dev)
         self.y = torch.empty((B, cfg.hidden), dtype=torch.float32, device=dev)
         self.prefill(stream)
+
+    def input_buffer(self) -> torch.Tensor:
+        """The device buffer holding q, k_new and v_new back to back (in that order)."""
+        return self._inbuf
 
     def prefill(self, stream=None):
         """Append every token but the last of each sequence (one call per sequence)."""
