@@ -102,3 +102,56 @@ def test_empty_batch_is_a_no_op(L):
     assert L.basiskv_route(ctypes.byref(cfg), ctypes.byref(good), 256, 0, 256, 256, None, None, 0, 256,
                            None) == bk.OK
     assert L.basiskv_out_proj(ctypes.byref(cfg), ctypes.byref(f), 256, 0, 256, None, 0, None) == bk.OK
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(rank_k=80), bk.ERR_UNSUPPORTED),             # residual rank above 64
+    (dict(rank_v=160, head_dim=128), bk.ERR_INVALID_ARG),  # latent rank above d
+    (dict(hidden=4100), bk.ERR_UNSUPPORTED),           # hidden not a multiple of 16
+    (dict(top_k=0), bk.ERR_INVALID_ARG),
+    (dict(num_kv_heads=0), bk.ERR_INVALID_ARG),
+])
+def test_more_config_limits(L, bad, status):
+    cfg = _cfg(**bad)
+    cache = bk.CCache(16, 16, 16, 16, 16, 16, 10, 10)
+    st = L.basiskv_route(ctypes.byref(cfg), ctypes.byref(cache), 16, 1, 16, 16, None, 16, 1 << 30, 16, None)
+    assert st == status
+
+
+def test_append_longer_than_the_block_table(L):
+    cfg = _cfg()
+    cache = bk.CCache(256, 256, 256, 256, 256, 256, 10, 4)      # 4 pages of 16 tokens
+    f = bk.CFactors(256, 256, 256, 256)
+    assert L.basiskv_append(ctypes.byref(cfg), ctypes.byref(cache), ctypes.byref(f), 256, 256, 1, 65, 256,
+                            None) == bk.ERR_INVALID_ARG
+    misaligned = bk.CFactors(264, 256, 256, 256)
+    assert L.basiskv_append(ctypes.byref(cfg), ctypes.byref(cache), ctypes.byref(misaligned), 256, 256, 1, 1,
+                            256, None) == bk.ERR_INVALID_ARG
+
+
+def test_out_proj_pointer_checks(L):
+    cfg = _cfg()
+    f = bk.CFactors(256, 256, 256, 256)
+    assert L.basiskv_out_proj(ctypes.byref(cfg), None, 256, 1, 256, None, 0, None) == bk.ERR_INVALID_ARG
+    assert L.basiskv_out_proj(ctypes.byref(cfg), ctypes.byref(bk.CFactors(256, 256, 256, 0)), 256, 1, 256, None,
+                              0, None) == bk.ERR_INVALID_ARG           # no fused factor
+    assert L.basiskv_out_proj(ctypes.byref(cfg), ctypes.byref(f), 260, 1, 256, None, 0, None) == bk.ERR_INVALID_ARG
+    assert L.basiskv_out_proj(ctypes.byref(cfg), ctypes.byref(f), 256, 1, None, None, 0, None) == bk.ERR_INVALID_ARG
+
+
+def test_workspace_grows_with_the_problem(L):
+    cfg = ctypes.byref(_cfg())
+    a = L.basiskv_workspace_bytes(cfg, 8, 2048)
+    assert L.basiskv_workspace_bytes(cfg, 16, 2048) > a
+    assert L.basiskv_workspace_bytes(cfg, 8, 4096) > a
+    assert L.basiskv_workspace_bytes(ctypes.byref(_cfg(dtype=bk.F32)), 8, 2048) > 0
+    assert L.basiskv_workspace_bytes(cfg, 8, 0) == 0
+    assert L.basiskv_workspace_bytes(cfg, -1, 2048) == 0
+
+
+def test_noalloc_refuses_shapes_beyond_its_scratch(L):
+    # 1024 sequences x 64 query heads need far more split scratch than the fixed 16 MiB
+    cfg = _cfg(num_q_heads=64, num_kv_heads=8, rank_v=128, top_k=256)
+    cache = bk.CCache(256, 256, 256, 256, 256, 256, 10, 4096)
+    st = L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(cache), 256, 1024, 256, 256, 256, 256, None)
+    assert st == bk.ERR_WORKSPACE
