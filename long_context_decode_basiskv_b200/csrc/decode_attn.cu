@@ -7,22 +7,24 @@
 // restricted to the selected tokens, with the weights applied to the rank-r
 // Value latents instead of full-width values.
 //
-// One launch: one CTA per (sequence, KV head, split of the union).  Each CTA
-// first merges the G query heads' selections into the ascending union of
-// pages with a G-bit head mask per page (a page chosen by several heads of a
-// group is read once) and keeps its split's slice of it.  Warp 0 is the
-//         producer: its lanes hold the split's union entries (page, mask,
-//         physical page, valid tokens) and lane 0 streams 16-token tiles (raw
-//         K rows and C rows, each contiguous in the page block) into a ring of
-//         shared-memory stages with 1-D bulk copies (cp.async.bulk, mbarrier
-//         completion, no multicast), writing each stage's head mask beside it.
-//         Warps 1..G are the consumers, one per query head of the group: a warp
-//         whose head selected the tile forms its 16 exact scores, updates an
-//         online softmax (running max and sum, base 2) and accumulates p * C;
-//         every consumer releases the stage.  Each head's split result (max,
-//         sum, acc[r]) goes to the workspace; the last CTA of a group to finish
-//         (counted with an atomic) merges the group's splits with the
-//         log-sum-exp rule and writes o_lat.
+// One launch: one CTA per (sequence, KV head, split of the union); the splits
+// fill one resident wave (decode_plan).  Each CTA first merges the G query
+// heads' selections into the ascending union of pages with a G-bit head mask
+// per page (a page chosen by several heads of a group is read once) and keeps
+// its split's equal share of it.  Two kernels stream the slice's 16-token
+// tiles (raw K rows and C rows, each contiguous in the page block) with 1-D
+// bulk copies (cp.async.bulk, mbarrier completion, bounded waits, no
+// multicast):
+//   * attn_mma_kernel (bf16, the main path): four warps per CTA, each with its
+//     own 3-slot ring, run all G heads of the group on the tensor cores
+//     (mma.sync m16n8k16: scores with heads as rows, online softmax in base
+//     2, P.C accumulated in registers); see the section below.
+//   * attn_kernel (fp32 and shapes without the swizzled layout): warp 0
+//     produces into a shared ring, warps 1..G consume, one per query head of
+//     the group, forming 16 exact scores per tile on the CUDA cores.
+// Each head's split result (max, sum, acc[r]) goes to the workspace; the last
+// CTA of a group to finish (counted with an atomic) merges the group's splits
+// with the log-sum-exp rule and writes o_lat.
 // HBM-bound: every byte of the union's pages is read once.
 #include "kernels.cuh"
 

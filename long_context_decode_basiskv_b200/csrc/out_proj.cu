@@ -6,10 +6,11 @@
 // so the rank-r attention output of each head is multiplied by the fused
 // factor G_h and the full Value width is never formed.
 //
-// Gt is stored [hidden][Hq][r]: row c is output column c for every (head,
-// latent dim), so y[b][c] is one dot product of length Hq*r per batch row.
-// This file holds the CUDA-core kernels: the fp32 (and small-batch) GEMV
-// path and the fp64 fusion that prepares Gt.
+// Gt holds row c = output column c for every (head, latent dim), so y[b][c]
+// is one dot product of length Hq*r per batch row.  This file holds the
+// CUDA-core kernels: the GEMV for fp32 (and for bf16 when Gt is not in the
+// tensor-core tile layout), and the fp64 fusion that writes Gt, tiled for the
+// tensor-core kernels when the shape allows.
 #include "kernels.cuh"
 
 namespace bkv {
