@@ -23,6 +23,15 @@ the plainest reading of those passages:
                   original keys, weights applied to the stored latents C
   5. out-proj     y = sum_h o_h G_h  with  G_h = B_g W_O,h
 
+A variant of step 3 routes once per KV group: the pages only say that routing
+picks key pages whose original keys are then read back (explainer, section
+"用Value潜变量辅助Key路由"), and under grouped-query attention the G query
+heads of a group share one cached key head (cloud.baidu.com article
+"大模型KV缓存压缩架构解析", section "1. 分组查询注意力（GQA）").  The variant
+scores page p for the whole group by the sum, or the maximum, over the group's
+heads of q_h . S_p and applies step 3's selection rule to that one score row;
+every head of the group then attends over the same pages.
+
 All arithmetic is fp64 numpy; a matmul is used as a library primitive where
 a step is a plain matrix product.  Rounding to the storage type (bf16
 round-to-nearest-even, or fp32) happens exactly where a value is stored.
@@ -40,7 +49,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "round_storage", "append_latents", "page_summaries", "route_pages",
+    "round_storage", "append_latents", "page_summaries", "route_pages", "route_pages_group",
     "sparse_attention", "fuse_out_factor", "out_projection",
     "SequenceCache", "prefill", "decode_step", "num_pages",
 ]
@@ -144,16 +153,40 @@ def route_pages(q, S, top_k: int):
     ascending order, fp64 scores of all n pages).
     """
     q = np.asarray(q, dtype=np.float64)
-    n = S.shape[0]
     scores = S @ q
+    return _select_pages(scores, top_k), scores
+
+
+def _select_pages(scores, top_k: int):
+    """Step 3's selection rule on one row of page scores (see route_pages)."""
+    n = scores.shape[0]
     if n <= top_k + 2:
-        return np.arange(n, dtype=np.int64), scores
+        return np.arange(n, dtype=np.int64)
     candidates = list(range(1, n - 1))
     candidates.sort(key=lambda p: (-scores[p], p))
     chosen = set(candidates[:top_k])
     chosen.add(0)
     chosen.add(n - 1)
-    return np.array(sorted(chosen), dtype=np.int64), scores
+    return np.array(sorted(chosen), dtype=np.int64)
+
+
+def route_pages_group(qs, S, top_k: int, reduce: str):
+    """Pages a whole KV group attends to: one selection for its G query heads.
+
+    qs: [G, d] the group's query rows; S: [n, d].  The group's score of page p
+    is the sum (reduce="sum") or the maximum (reduce="max") over the heads h
+    of q_h . S_p; step 3's rule then selects from that one row.  Returns
+    (selected pages in ascending order, fp64 group scores of all n pages).
+    """
+    qs = np.asarray(qs, dtype=np.float64)
+    per_head = S @ qs.T  # [n, G]
+    if reduce == "sum":
+        scores = per_head.sum(axis=1)
+    elif reduce == "max":
+        scores = per_head.max(axis=1)
+    else:
+        raise ValueError(f"reduce must be 'sum' or 'max', not {reduce!r}")
+    return _select_pages(scores, top_k), scores
 
 
 # --------------------------------------------------------------------------
@@ -260,13 +293,16 @@ def prefill(keys, values, A, P, E, page_size, storage, capacity=None):
     return cache
 
 
-def decode_step(cache: SequenceCache, k_new, v_new, q, A, P, E, G, top_k: int):
+def decode_step(cache: SequenceCache, k_new, v_new, q, A, P, E, G, top_k: int, routing: str = "head"):
     """One decode step of one sequence: append, summary, route, attend, project.
 
     k_new, v_new: [Hkv, d] (the new token); q: [Hq, d]; G: [Hq, r, hidden].
+    routing: "head" (one selection per query head), or "group_sum" /
+    "group_max" (one selection per KV group, see route_pages_group).
     Returns a dict with per-head selections ``sel`` (list of arrays),
-    routing ``scores`` (list), latent outputs ``o_lat`` [Hq, r], the softmax
-    weight sums and the output ``y`` [hidden].
+    routing ``scores`` (list: per head, or per KV group in the group modes),
+    latent outputs ``o_lat`` [Hq, r], the softmax weight sums and the output
+    ``y`` [hidden].
     """
     cache.append(np.asarray(k_new)[None], np.asarray(v_new)[None], A, P, E)
     Hq = q.shape[0]
@@ -274,13 +310,24 @@ def decode_step(cache: SequenceCache, k_new, v_new, q, A, P, E, G, top_k: int):
     group = Hq // Hkv
     L, n = cache.length, cache.pages
     sels, scores, wsum = [], [], []
+    if routing not in ("head", "group_sum", "group_max"):
+        raise ValueError(f"unknown routing {routing!r}")
+    group_sel = []
+    if routing != "head":
+        for g in range(Hkv):
+            gsel, gsc = route_pages_group(q[g * group:(g + 1) * group], cache.S[g, :n], top_k, routing[6:])
+            group_sel.append(gsel)
+            scores.append(gsc)
     o_lat = np.zeros((Hq, cache.C.shape[2]))
     for h in range(Hq):
         g = h // group
-        sel, sc = route_pages(q[h], cache.S[g, :n], top_k)
+        if routing == "head":
+            sel, sc = route_pages(q[h], cache.S[g, :n], top_k)
+            scores.append(sc)
+        else:
+            sel = group_sel[g]
         o, w, _ = sparse_attention(q[h], cache.K[g, :L], cache.C[g, :L], sel, cache.page_size)
         sels.append(sel)
-        scores.append(sc)
         wsum.append(w.sum())
         o_lat[h] = o
     y = out_projection(o_lat, G)

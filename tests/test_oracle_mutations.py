@@ -13,7 +13,7 @@ from oracle import basiskv_oracle as ORACLE
 from tests.test_oracle_pins import ALL_CHECKS
 
 _orig = {name: getattr(ORACLE, name) for name in
-         ["append_latents", "page_summaries", "route_pages", "sparse_attention",
+         ["append_latents", "page_summaries", "route_pages", "route_pages_group", "sparse_attention",
           "fuse_out_factor", "out_projection", "round_storage", "_round_bf16"]}
 
 
@@ -102,6 +102,22 @@ def _fuse_transposed_wo(Bf, W_O, num_q_heads, storage):
     return _orig["fuse_out_factor"](Bf, Wt, num_q_heads, storage)
 
 
+def _group_first_head_only(qs, S, top_k, reduce):
+    return _orig["route_pages_group"](np.asarray(qs)[:1], S, top_k, reduce)
+
+
+def _group_max_as_min(qs, S, top_k, reduce):
+    if reduce != "max":
+        return _orig["route_pages_group"](qs, S, top_k, reduce)
+    sc = (S @ np.asarray(qs, np.float64).T).min(axis=1)
+    return ORACLE._select_pages(sc, top_k), sc
+
+
+def _group_sum_as_mean(qs, S, top_k, reduce):
+    sel, sc = _orig["route_pages_group"](qs, S, top_k, reduce)
+    return sel, (sc / len(qs) if reduce == "sum" else sc)
+
+
 def _outproj_first_head_only(o_lat, G):
     return o_lat[0] @ G[0]
 
@@ -123,6 +139,9 @@ MUTATIONS = {
     "route_tie_prefers_high_index": ("route_pages", _route_tie_high_index),
     "route_picks_lowest_scores": ("route_pages", _route_lowest),
     "route_keeps_one_too_many": ("route_pages", _route_k_plus_one),
+    "group_route_first_head_only": ("route_pages_group", _group_first_head_only),
+    "group_route_max_as_min": ("route_pages_group", _group_max_as_min),
+    "group_route_sum_as_mean": ("route_pages_group", _group_sum_as_mean),
     "attention_missing_sqrt_d": ("sparse_attention", _attn_no_scale),
     "attention_skips_partial_page": ("sparse_attention", _attn_skip_partial_page),
     "fuse_wrong_head_group": ("fuse_out_factor", _fuse_wrong_group),

@@ -210,6 +210,59 @@ def check_route_small_n(o):
     np.testing.assert_array_equal(sel, [0, 3, 4])
 
 
+def check_route_group_worked_example(o):
+    """Two heads reading one coordinate each; the group scores worked by hand.
+
+    Per page (1..4) the head scores are (5, -9), (-9, 4), (1, 1), (3, 3):
+    max over heads = 5, 4, 1, 3 and sum = -4, -5, 2, 6.  With k = 2 the max
+    keeps pages 1 and 2, the sum pages 3 and 4 (head 0 alone would keep 1 and 4).
+    """
+    S = np.array([[0.0, 0], [5, -9], [-9, 4], [1, 1], [3, 3], [0, 0]])
+    qs = np.eye(2)
+    sel, sc = o.route_pages_group(qs, S, 2, "max")
+    np.testing.assert_array_equal(sel, [0, 1, 2, 5])
+    np.testing.assert_allclose(sc[1:5], [5, 4, 1, 3], atol=0)
+    sel, sc = o.route_pages_group(qs, S, 2, "sum")
+    np.testing.assert_array_equal(sel, [0, 3, 4, 5])
+    np.testing.assert_allclose(sc[1:5], [-4, -5, 2, 6], atol=0)
+    np.testing.assert_array_equal(o.route_pages(qs[0], S, 2)[0], [0, 1, 4, 5])
+
+
+def check_route_group_reductions(o):
+    """Group routing against identities: one head is per-head routing; the sum
+    is the score of the summed query (linearity); identical heads select what
+    one of them selects; the max is at least every head's score."""
+    rng = np.random.default_rng(11)
+    for n, k, G in [(64, 8, 4), (300, 17, 8), (12, 3, 2), (9, 8, 4)]:
+        S = rng.standard_normal((n, 16))
+        qs = rng.standard_normal((G, 16))
+        for red in ("sum", "max"):
+            sel1, sc1 = o.route_pages_group(qs[:1], S, k, red)
+            sel_h, sc_h = o.route_pages(qs[0], S, k)
+            np.testing.assert_array_equal(sel1, sel_h)
+            np.testing.assert_allclose(sc1, sc_h, atol=1e-12)
+            same = np.repeat(qs[:1], G, axis=0)
+            np.testing.assert_array_equal(o.route_pages_group(same, S, k, red)[0], sel_h)
+        sel, sc = o.route_pages_group(qs, S, k, "sum")
+        qsum = qs.sum(axis=0)
+        np.testing.assert_allclose(sc, S @ qsum, atol=1e-11)
+        np.testing.assert_array_equal(sel, _sort_reference(S @ qsum, k))
+        sel, sc = o.route_pages_group(qs, S, k, "max")
+        for h in range(G):
+            assert np.all(sc >= S @ qs[h] - 1e-12)
+        assert np.all(np.isclose(sc[:, None], S @ qs.T, atol=1e-12).any(axis=1))  # attained by a head
+        np.testing.assert_array_equal(sel, _sort_reference(sc, k))
+        assert len(sel) == min(n, k + 2)
+
+
+def test_route_group_worked_example():
+    check_route_group_worked_example(ORACLE)
+
+
+def test_route_group_reductions():
+    check_route_group_reductions(ORACLE)
+
+
 def test_route_full_sort():
     check_route_full_sort(ORACLE)
 
@@ -354,6 +407,41 @@ def check_new_token_is_attended(o):
     np.testing.assert_allclose(out["o_lat"][0], V[-1, 0], atol=1e-6)
 
 
+def check_decode_group_routing(o):
+    """Group routing in a decode step: with every page selected it is dense GQA
+    attention; with few pages every head of a group attends, by textbook
+    softmax, over the tokens of the pages its group's summed or max score
+    keeps (computed here from the summed query and an elementwise maximum)."""
+    rng = np.random.default_rng(15)
+    Hq, Hkv, d, ps, T, hid = 4, 2, 8, 4, 41, 5
+    G_ = Hq // Hkv
+    K, V = _tiny_sequence(rng, T, Hkv, d)
+    q = rng.standard_normal((Hq, d))
+    eye = np.stack([np.eye(d)] * Hkv)
+    W_O = rng.standard_normal((Hq * d, hid))
+    G = o.fuse_out_factor(eye, W_O, Hq, "f64")
+    n = o.num_pages(T, ps)
+    for routing in ("group_sum", "group_max"):
+        cache = o.prefill(K[:-1], V[:-1], eye, eye, eye, ps, "f64", capacity=T)
+        out = o.decode_step(cache, K[-1], V[-1], q, eye, eye, eye, G, top_k=100, routing=routing)
+        heads = [_sdpa(q[h], K[:, h // G_], V[:, h // G_]) for h in range(Hq)]
+        np.testing.assert_allclose(out["y"], np.concatenate(heads) @ W_O, atol=1e-11)
+        cache = o.prefill(K[:-1], V[:-1], eye, eye, eye, ps, "f64", capacity=T)
+        out = o.decode_step(cache, K[-1], V[-1], q, eye, eye, eye, G, top_k=3, routing=routing)
+        for g in range(Hkv):
+            Sg = cache.S[g, :n]  # the stored (fp32) summaries: with E = I, the mean key of each page
+            mean_k = np.stack([K[p * ps:(p + 1) * ps, g].mean(axis=0) for p in range(n)])
+            np.testing.assert_allclose(Sg, mean_k, rtol=1e-6, atol=1e-6)
+            qg = q[g * G_:(g + 1) * G_]
+            gs = Sg @ qg.sum(axis=0) if routing == "group_sum" else np.maximum.reduce(Sg @ qg.T, axis=1)
+            np.testing.assert_allclose(out["scores"][g], gs, atol=1e-12)
+            want = _sort_reference(gs, 3)
+            for h in range(g * G_, (g + 1) * G_):
+                np.testing.assert_array_equal(out["sel"][h], want)
+                tok = np.concatenate([np.arange(p * ps, min(T, (p + 1) * ps)) for p in want])
+                np.testing.assert_allclose(out["o_lat"][h], _sdpa(q[h], K[tok, g], V[tok, g]), atol=1e-12)
+
+
 def check_golden(o):
     with open(GOLDEN) as f:
         gx = json.load(f)
@@ -395,6 +483,10 @@ def test_new_token_is_attended():
     check_new_token_is_attended(ORACLE)
 
 
+def test_decode_group_routing():
+    check_decode_group_routing(ORACLE)
+
+
 def test_golden_worked_example():
     check_golden(ORACLE)
 
@@ -424,6 +516,7 @@ ALL_CHECKS = [
     check_bf16_rounding, check_append_identity, check_append_projection,
     check_summary_closed_form, check_summary_low_rank_residual,
     check_route_full_sort, check_route_ties, check_route_bruteforce, check_route_small_n,
+    check_route_group_worked_example, check_route_group_reductions, check_decode_group_routing,
     check_attention_dense_reduction, check_attention_subset,
     check_out_projection_associativity, check_decode_dense_special_case,
     check_decode_all_pages_real_factors, check_new_token_is_attended, check_golden,
