@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="llama3_8b_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--routing", default="head", choices=["head", "group_sum", "group_max"],
+                    help="one page selection per query head (the method as stated), or per KV group")
     ap.add_argument("--oracle-seqs", type=int, default=2, help="sequences in the CPU-baseline sample")
     ap.add_argument("--oracle-repeats", type=int, default=100,
                     help="decode steps per sampled sequence in the CPU baseline (about 10 s in total)")
@@ -171,6 +173,7 @@ def algorithmic_bytes(eng):
     pages = [-(-L // P) for L in case.lengths]
     sel = eng.sel.cpu().numpy()
     cnt = eng.sel_cnt.cpu().numpy()
+    score_rows = Hq if eng.routing == "head" else Hkv
     union = 0
     for b in range(B):
         for g in range(Hkv):
@@ -180,7 +183,7 @@ def algorithmic_bytes(eng):
             union += len(u)
     q_bytes = B * Hq * d * es
     sel_bytes = B * Hq * (k + 2) * 4
-    route = sum(pages) * Hkv * d * 4 + 2 * sum(pages) * Hq * 4 + q_bytes + sel_bytes
+    route = sum(pages) * Hkv * d * 4 + 2 * sum(pages) * score_rows * 4 + q_bytes + sel_bytes
     decode = union * P * (d + r) * es + q_bytes + sel_bytes + B * Hq * r * 4
     out = Hq * r * wl.hidden * es + B * Hq * r * 4 + B * wl.hidden * 4
     append = B * Hkv * ((2 * d * r + d * s) * es + 2 * d * es + P * (r + s) * es + d * 4)
@@ -215,7 +218,7 @@ def profiled_traffic(kernel_file: str):
 # ---------------------------------------------------------------------------
 # CPU baseline: the oracle on a bounded sample
 # ---------------------------------------------------------------------------
-def oracle_sample(case, nseq: int, repeats: int = 1):
+def oracle_sample(case, nseq: int, repeats: int = 1, routing: str = "head"):
     """Time the oracle's decode step (append .. out-projection) on `nseq` sequences.
 
     The prefill of each sequence's oracle cache is untimed.  A repeat re-runs
@@ -244,9 +247,9 @@ def oracle_sample(case, nseq: int, repeats: int = 1):
             for _ in range(repeats):
                 cache.length = L - 1
                 t0 = time.perf_counter()
-                O.decode_step(cache, K[-1], V[-1], q, A, P, E, G, wl.top_k)
+                O.decode_step(cache, K[-1], V[-1], q, A, P, E, G, wl.top_k, routing=routing)
                 times.append(time.perf_counter() - t0)
-    desc = (f"fp64 numpy oracle, 1 thread: decode step (append, summary, route, attention, "
+    desc = (f"fp64 numpy oracle, 1 thread: decode step (append, summary, {routing} route, attention, "
             f"out-projection) of {min(nseq, wl.batch)} of the {wl.batch} sequences x {repeats}, "
             f"prefill untimed")
     return times, desc
@@ -265,7 +268,7 @@ def run_ours(args, world, rank, local):
     case = make_case(wl, dev)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
-        eng = DecodeEngine(case, device=dev)
+        eng = DecodeEngine(case, device=dev, routing=args.routing)
         eng.step()
     torch.cuda.synchronize()
     if int(eng.err.item()) != 0:
@@ -323,7 +326,8 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = measured_peak()
     attn_gbs = nbytes["decode_attn"] / (mean["decode_attn"] * 1e-3) / 1e9
     ra_gbs = (nbytes["route"] + nbytes["decode_attn"]) / ((mean["append_route"] + mean["decode_attn"]) * 1e-3) / 1e9
-    traffic_rec = profiled_traffic("decode_attn.cu")
+    # the committed counters are for per-head routing (other routings read other pages)
+    traffic_rec = profiled_traffic("decode_attn.cu") if args.routing == "head" else None
     roofline = {
         "kernel": "basiskv_decode_attn (one launch: union slice, attention, split merge)",
         "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
@@ -369,7 +373,7 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, desc = oracle_sample(case, args.oracle_seqs, args.oracle_repeats)
+        times, desc = oracle_sample(case, args.oracle_seqs, args.oracle_repeats, args.routing)
         cpu = {"value": round(len(times) / sum(times), 3), "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": desc, "seconds": round(sum(times), 3)}
 
@@ -382,7 +386,8 @@ def run_ours(args, world, rank, local):
             "config": {"workload": wl.name, "batch": wl.batch, "context": wl.context if not wl.ragged else list(wl.ragged),
                        "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                        "page_size": wl.page_size, "rank_v": wl.rank_v, "rank_k": wl.rank_k,
-                       "top_k": wl.top_k, "hidden": wl.hidden, "parallelism": f"replicas x{world}",
+                       "top_k": wl.top_k, "hidden": wl.hidden, "routing": args.routing,
+                       "parallelism": f"replicas x{world}",
                        "l2": "flushed between steps (read of a 256 MiB buffer)",
                        "timing": "one CUDA graph per step (append || route on forked streams, decode_attn, out_proj), CUDA events around each replay; kernels_us from per-phase graphs in a separate pass; route+attn GB/s counts the append || route phase time"},
             "kernels_us": {k: round(v * 1e3, 2) for k, v in mean.items()},
@@ -409,7 +414,7 @@ def run_reference(args, world, rank):
         return
     wl = WORKLOADS[args.workload]
     case = make_case(wl, "cpu")
-    times, desc = oracle_sample(case, 1, repeats=args.warmup + args.steps)
+    times, desc = oracle_sample(case, 1, repeats=args.warmup + args.steps, routing=args.routing)
     timed = times[args.warmup:]
     value = len(timed) / sum(timed)
     line = {
@@ -417,7 +422,8 @@ def run_reference(args, world, rank):
         "warmup": args.warmup, "ms_per_step": round(1e3 * sum(timed) / len(timed), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
-        "config": {"workload": wl.name, "batch": wl.batch, "sample": "one sequence per step"},
+        "config": {"workload": wl.name, "batch": wl.batch, "routing": args.routing,
+                   "sample": "one sequence per step"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

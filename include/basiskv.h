@@ -9,6 +9,7 @@
  *   basiskv_route        (step 3)   score every page of every sequence for every
  *                        query head against the summaries; keep the top-k pages
  *                        plus the sink page and the recent page
+ *                        (basiskv_route_group: one selection per KV group)
  *   basiskv_decode_attn  (step 4)   exact attention of each query head over the
  *                        original keys of its selected pages, accumulating the
  *                        Value latents (rank-r output per head)
@@ -68,6 +69,9 @@ typedef enum {
 } basiskv_status;
 
 typedef enum { BASISKV_F32 = 0, BASISKV_BF16 = 1 } basiskv_dtype;
+
+/* How basiskv_route_group folds the scores of a KV group's query heads. */
+typedef enum { BASISKV_GROUP_SUM = 1, BASISKV_GROUP_MAX = 2 } basiskv_group_reduce;
 
 /* Bits OR-ed into *err_flag by the kernels. */
 #define BASISKV_DEVERR_BLOCK_TABLE 1   /* block_table entry outside [0, num_phys_pages)      */
@@ -180,6 +184,28 @@ BASISKV_API basiskv_status basiskv_route(const basiskv_config* cfg, const basisk
                              const void* q, int32_t batch, int32_t* sel, int32_t* sel_cnt,
                              float* scores, void* workspace, size_t workspace_bytes,
                              int32_t* err_flag, void* stream);
+
+/*
+ * Step 3, per-KV-group variant.  The pages say only that routing picks key
+ * pages whose original keys are then read (kongchang.com explainer, section
+ * "用Value潜变量辅助Key路由"); under grouped-query attention the G = Hq/Hkv
+ * query heads of a group share one key head (cloud.baidu.com article
+ * "大模型KV缓存压缩架构解析", section "1. 分组查询注意力（GQA）").  This
+ * call routes once per (sequence, KV group g): the group score of page p is
+ * the sum (reduce = BASISKV_GROUP_SUM) or the maximum (BASISKV_GROUP_MAX,
+ * a NaN head score wins) over h = gG .. gG+G-1 of q_h . S_p in fp32, and the
+ * selection rule of basiskv_route is applied to that one row.  The pages are
+ * written to the sel / sel_cnt rows of all G heads of the group, in
+ * basiskv_route's layout, so basiskv_decode_attn reads top_k + 2 pages per
+ * group (instead of the union of G per-head selections).
+ * scores (device, optional): [batch][Hkv][max_pages] fp32 group scores.
+ * Other arguments, concurrency and workspace as for basiskv_route.  Any other
+ * value of `reduce` is BASISKV_ERR_INVALID_ARG.
+ */
+BASISKV_API basiskv_status basiskv_route_group(const basiskv_config* cfg, const basiskv_cache* cache,
+                                   const void* q, int32_t batch, int32_t reduce, int32_t* sel,
+                                   int32_t* sel_cnt, float* scores, void* workspace,
+                                   size_t workspace_bytes, int32_t* err_flag, void* stream);
 
 /*
  * Step 4.  Exact sparse attention.  For each (b, h): over the valid tokens j

@@ -19,13 +19,14 @@ LIB_PATH = os.path.join(_HERE, "libbasiskv.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
+GROUP_SUM, GROUP_MAX = 1, 2
 DEVERR_BLOCK_TABLE, DEVERR_SELECTION, DEVERR_SEQ_LEN, DEVERR_TIMEOUT, DEVERR_WORKSPACE = 1, 2, 4, 8, 16
 
 # every function include/basiskv.h declares
 SYMBOLS = [
     "basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
     "basiskv_fuse_out_factor", "basiskv_workspace_bytes", "basiskv_status_string",
-    "basiskv_abi_version", "basiskv_decode_attn_noalloc",
+    "basiskv_abi_version", "basiskv_decode_attn_noalloc", "basiskv_route_group",
 ]
 
 
@@ -63,6 +64,7 @@ def lib():
     pc, pk, pf = ctypes.POINTER(CConfig), ctypes.POINTER(CCache), ctypes.POINTER(CFactors)
     L.basiskv_append.argtypes = [pc, pk, pf, vp, vp, i32, i32, vp, vp]
     L.basiskv_route.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, sz, vp, vp]
+    L.basiskv_route_group.argtypes = [pc, pk, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp]
     L.basiskv_decode_attn.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, sz, vp, vp]
     L.basiskv_out_proj.argtypes = [pc, pf, vp, i32, vp, vp, sz, vp]
     L.basiskv_decode_attn_noalloc.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, vp]
@@ -73,7 +75,8 @@ def lib():
     L.basiskv_status_string.restype = ctypes.c_char_p
     L.basiskv_abi_version.argtypes = []
     for name in ["basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
-                 "basiskv_fuse_out_factor", "basiskv_abi_version", "basiskv_decode_attn_noalloc"]:
+                 "basiskv_fuse_out_factor", "basiskv_abi_version", "basiskv_decode_attn_noalloc",
+                 "basiskv_route_group"]:
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -217,6 +220,24 @@ def route(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor, se
     _check(lib().basiskv_route(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), _ptr(q), B, _ptr(sel),
                                _ptr(sel_cnt), _ptr(scores), _ptr(ws), ws.numel(), _ptr(err),
                                _stream(stream)), "basiskv_route")
+
+
+def route_group(cfg: Config, cache: PagedCache, q: torch.Tensor, reduce: int, sel: torch.Tensor,
+                sel_cnt: torch.Tensor, ws: torch.Tensor, err: torch.Tensor,
+                scores: Optional[torch.Tensor] = None, stream=None):
+    """One selection per KV group (reduce = GROUP_SUM or GROUP_MAX of its heads' scores),
+    written to the sel rows of every head of the group; scores [B][Hkv][max_pages]."""
+    B = q.shape[0]
+    _need(q, "q", cfg.dtype, (B, cfg.num_q_heads, cfg.head_dim))
+    _need(sel, "sel", torch.int32, (B, cfg.num_q_heads, cfg.top_k + 2))
+    _need(sel_cnt, "sel_cnt", torch.int32, (B, cfg.num_q_heads))
+    _need(ws, "workspace", torch.uint8)
+    _need(err, "err", torch.int32)
+    if scores is not None:
+        _need(scores, "scores", torch.float32, (B, cfg.num_kv_heads, cache.max_pages))
+    _check(lib().basiskv_route_group(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), _ptr(q), B, reduce,
+                                     _ptr(sel), _ptr(sel_cnt), _ptr(scores), _ptr(ws), ws.numel(),
+                                     _ptr(err), _stream(stream)), "basiskv_route_group")
 
 
 def decode_attn(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor,

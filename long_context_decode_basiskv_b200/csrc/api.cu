@@ -125,9 +125,9 @@ basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* ca
   return cuda_status(launch_append(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
 }
 
-basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
-                             int32_t batch, int32_t* sel, int32_t* sel_cnt, float* scores,
-                             void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+static basiskv_status route_common(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
+                                   int32_t batch, int group_mode, int32_t* sel, int32_t* sel_cnt, float* scores,
+                                   void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
   basiskv_status s = check_config(cfg);
   if (s != BASISKV_OK) return s;
   if ((s = check_cache(cfg, cache, false)) != BASISKV_OK) return s;
@@ -140,8 +140,21 @@ basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cac
   float* sc = scores ? scores : reinterpret_cast<float*>(wsb + w.scores);
   RouteParams rp{q, cache->summary, cache->block_table, cache->seq_len, sc, sel, sel_cnt, err_flag,
                  batch, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cache->max_pages,
-                 cache->num_phys_pages, cfg->top_k, scores ? 1 : 0};
+                 cache->num_phys_pages, cfg->top_k, scores ? 1 : 0, group_mode};
   return cuda_status(launch_route(rp, cfg->head_dim, cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream));
+}
+
+basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
+                             int32_t batch, int32_t* sel, int32_t* sel_cnt, float* scores,
+                             void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+  return route_common(cfg, cache, q, batch, 0, sel, sel_cnt, scores, ws, ws_bytes, err_flag, stream);
+}
+
+basiskv_status basiskv_route_group(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
+                                   int32_t batch, int32_t reduce, int32_t* sel, int32_t* sel_cnt,
+                                   float* scores, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+  if (reduce != BASISKV_GROUP_SUM && reduce != BASISKV_GROUP_MAX) return BASISKV_ERR_INVALID_ARG;
+  return route_common(cfg, cache, q, batch, reduce, sel, sel_cnt, scores, ws, ws_bytes, err_flag, stream);
 }
 
 basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,

@@ -29,12 +29,14 @@ struct RouteParams {
   const float* summary;
   const int32_t* block_table;
   const int32_t* seq_len;
-  float* scores;    // [B][Hq][max_pages]
+  float* scores;    // [B][Hq][max_pages] per head; [B][Hkv][max_pages] per group
   int32_t* sel;     // [B][Hq][top_k + 2]
   int32_t* sel_cnt; // [B][Hq]
   int32_t* err;
   int batch, Hq, Hkv, page, max_pages, num_phys, top_k;
   int all_pages;    // 0: skip the sink and recent pages (always kept; their scores are not needed)
+  int group_mode;   // 0: one selection per query head; 1 / 2: one per KV group from the
+                    // sum / maximum of its heads' scores, copied to every head of the group
 };
 cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st);
 

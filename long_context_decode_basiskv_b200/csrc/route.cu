@@ -26,6 +26,13 @@
 //     the lowest page indices; two block scans (ties, kept pages) give every
 //     thread its output positions, so sel is written in ascending page order.
 // The result is the same as sorting by (score descending, page ascending).
+//
+// Per-group routing (group_mode 1 / 2): the score kernel folds the G head
+// scores of a page, which sit on neighbouring lanes after the transpose
+// reduction, into their sum or maximum and writes one row per (sequence, KV
+// group); one selection CTA per group ranks it and writes its pages to the
+// sel rows of all G heads, so the attention kernel reads k + 2 pages per
+// group.
 #include "kernels.cuh"
 
 namespace bkv {
@@ -35,6 +42,12 @@ constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kScoreWarpPages = 32;
 constexpr int kScoreCtaPages = kScoreWarps * kScoreWarpPages;
+
+// sum (mode 1) or maximum (mode 2) of two head scores; the maximum keeps a NaN
+__device__ __forceinline__ float group_fold(float a, float b, int mode) {
+  if (mode == 1) return a + b;
+  return (a > b || a != a) ? a : b;
+}
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_kernel(RouteParams p) {
@@ -74,6 +87,7 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
 #pragma unroll
     for (int u = 0; u < DPL; ++u) qf[hi][u] = sq[hi * D + lane * DPL + u];
   float* outb = p.scores + qrow * p.max_pages;
+  float* outg = p.scores + ((size_t)b * p.Hkv + g) * p.max_pages;  // the group's row (group modes)
 #pragma unroll 1
   for (int i0 = 0; i0 < kScoreWarpPages; i0 += kPagesPerWarp) {
     const int p0 = pw0 + i0;
@@ -108,7 +122,29 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
       }
     transpose_reduce<N>(part, lane);
     float* out = outb + p0;
-    if constexpr (N <= 32) {
+    if (p.group_mode != 0) {
+      // the G head scores of page i: N <= 32, lanes [i G kDup, (i + 1) G kDup)
+      // hold one each (kDup copies); N = 64, lanes [i G / 2, (i + 1) G / 2) two each
+      float v;
+      int i;
+      bool writer;
+      if constexpr (N <= 32) {
+        constexpr int kDup = 32 / N;
+        v = part[0];
+#pragma unroll
+        for (int o = kDup; o < kDup * G; o <<= 1) v = group_fold(v, __shfl_xor_sync(kFull, v, o), p.group_mode);
+        i = lane / (kDup * G);
+        writer = lane % (kDup * G) == 0;
+      } else {
+        v = group_fold(part[0], part[1], p.group_mode);
+#pragma unroll
+        for (int o = 1; o < G / 2; o <<= 1) v = group_fold(v, __shfl_xor_sync(kFull, v, o), p.group_mode);
+        i = lane / (G / 2);
+        writer = lane % (G / 2) == 0;
+      }
+      const int ph = __shfl_sync(kFull, my_phys, i0 + i);
+      if (writer && p0 + i < n && ph != -1) outg[p0 + i] = (ph == -2) ? -INFINITY : v;
+    } else if constexpr (N <= 32) {
       constexpr int kDup = 32 / N;
       const int idx = lane / kDup;
       const int i = idx / G, hi = idx % G;
@@ -155,24 +191,48 @@ __device__ __forceinline__ int block_total(int v, int* red, int& phase) {
   return t;
 }
 
+// The score row a selection CTA (x = blockIdx.x) ranks and the sel rows it
+// writes: its own head's, or the G heads' of its group (contiguous rows).
+struct SelRows {
+  size_t in, out;
+  int copies;
+};
+__device__ __forceinline__ SelRows sel_rows(const RouteParams& p, int x, int b) {
+  if (p.group_mode == 0) {
+    const size_t r = (size_t)b * p.Hq + x;
+    return {r, r, 1};
+  }
+  const int G = p.Hq / p.Hkv;
+  return {(size_t)b * p.Hkv + x, (size_t)b * p.Hq + (size_t)x * G, G};
+}
+
+// sel entry i of every output row of the CTA
+__device__ __forceinline__ void put_sel(const RouteParams& p, const SelRows& r, int i, int32_t v) {
+  int32_t* out = p.sel + r.out * (p.top_k + 2) + i;
+  for (int c = 0; c < r.copies; ++c) out[(size_t)c * (p.top_k + 2)] = v;
+}
+
+__device__ __forceinline__ void put_cnt(const RouteParams& p, const SelRows& r, int v) {
+  for (int c = 0; c < r.copies; ++c) p.sel_cnt[r.out + c] = v;
+}
+
 template <int KPT>
 __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
   __shared__ int red[2 * kSelectWarps];
   __shared__ int warp_tot[32];
   allow_dependents();  // the attention kernel may launch; it waits for this selection
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int b = blockIdx.y, tid = threadIdx.x;
   const int L = p.seq_len[b];
   const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
   const int kk = p.top_k;
-  const size_t row = (size_t)b * p.Hq + h;
-  int32_t* out = p.sel + row * (kk + 2);
+  const SelRows rows = sel_rows(p, blockIdx.x, b);
   if (n <= kk + 2) {
-    for (int i = tid; i < kk + 2; i += kSelectThreads) out[i] = (i < n) ? i : -1;
-    if (tid == 0) p.sel_cnt[row] = n;
+    for (int i = tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, (i < n) ? i : -1);
+    if (tid == 0) put_cnt(p, rows, n);
     return;
   }
   // thread t holds pages [t * KPT, t * KPT + KPT)
-  const float* sc = p.scores + row * p.max_pages;
+  const float* sc = p.scores + rows.in * p.max_pages;
   const int p0 = tid * KPT;
   uint32_t key[KPT];
 #pragma unroll
@@ -231,9 +291,9 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParam
   int pos = block_exclusive_scan(kept, warp_tot, total);
 #pragma unroll
   for (int j = 0; j < KPT; ++j)
-    if (take[j]) out[pos++] = p0 + j;
-  for (int i = total + tid; i < kk + 2; i += kSelectThreads) out[i] = -1;
-  if (tid == 0) p.sel_cnt[row] = total;
+    if (take[j]) put_sel(p, rows, pos++, p0 + j);
+  for (int i = total + tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, -1);
+  if (tid == 0) put_cnt(p, rows, total);
 }
 
 // ---------------------------------------------------------------------------
@@ -295,18 +355,17 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(Route
   __shared__ float s_T;
   allow_dependents();
 
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int b = blockIdx.y;
   const int tid = threadIdx.x;
   const int L = p.seq_len[b];
   const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
   const int kk = p.top_k;
-  const size_t row = (size_t)b * p.Hq + h;
-  int32_t* out = p.sel + row * (kk + 2);
-  const float* sc = p.scores + row * p.max_pages;
+  const SelRows rows = sel_rows(p, blockIdx.x, b);
+  const float* sc = p.scores + rows.in * p.max_pages;
 
   if (n <= kk + 2) {
-    for (int i = tid; i < kk + 2; i += blockDim.x) out[i] = (i < n) ? i : -1;
-    if (tid == 0) p.sel_cnt[row] = n;
+    for (int i = tid; i < kk + 2; i += blockDim.x) put_sel(p, rows, i, (i < n) ? i : -1);
+    if (tid == 0) put_cnt(p, rows, n);
     return;
   }
   const int ncand = n - 2;  // pages 1 .. n-2 compete
@@ -460,11 +519,11 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(Route
         take = v > T || (v == T && er < keep_eq);
         if (v == T) ++er;
       }
-      if (take) out[pos++] = pg;
+      if (take) put_sel(p, rows, pos++, pg);
     }
   }
-  for (int i = tot + tid; i < kk + 2; i += blockDim.x) out[i] = -1;
-  if (tid == 0) p.sel_cnt[row] = tot;
+  for (int i = tot + tid; i < kk + 2; i += blockDim.x) put_sel(p, rows, i, -1);
+  if (tid == 0) put_cnt(p, rows, tot);
 }
 
 
@@ -494,7 +553,7 @@ cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cu
   else
     e = (d == 128) ? launch_score_g<float, 128>(p, G, st) : launch_score_g<float, 64>(p, G, st);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.Hq, p.batch);
+  const dim3 grid(p.group_mode ? p.Hkv : p.Hq, p.batch);
   if (p.max_pages <= kSelectThreads * 8) {
     route_select_kernel<8><<<grid, kSelectThreads, 0, st>>>(p);
   } else if (p.max_pages <= kSelectThreads * 16) {

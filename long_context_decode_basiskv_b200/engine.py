@@ -4,7 +4,9 @@
 the library's own append kernel in prefill mode), the factors with the fused
 out-projection factor (built by the library's fusion kernel), the step's
 inputs and outputs, and one workspace.  ``step()`` enqueues the four calls of
-one decode step: append, route, decode_attn, out_proj.
+one decode step: append, route, decode_attn, out_proj.  ``routing`` picks one
+selection per query head ("head") or per KV group from the sum ("group_sum")
+or maximum ("group_max") of its heads' page scores.
 """
 from __future__ import annotations
 
@@ -20,8 +22,14 @@ def config_of(case: Case) -> bk.Config:
                      wl.page_size, wl.hidden, wl.top_k, wl.torch_dtype)
 
 
+_GROUP_REDUCE = {"group_sum": bk.GROUP_SUM, "group_max": bk.GROUP_MAX}
+
+
 class DecodeEngine:
-    def __init__(self, case: Case, device="cuda", stream=None):
+    def __init__(self, case: Case, device="cuda", stream=None, routing: str = "head"):
+        if routing != "head" and routing not in _GROUP_REDUCE:
+            raise ValueError(f"routing must be 'head', 'group_sum' or 'group_max', not {routing!r}")
+        self.routing = routing
         self.case = case
         self.cfg = cfg = config_of(case)
         self.device = torch.device(device)
@@ -83,7 +91,11 @@ class DecodeEngine:
         bk.append(self.cfg, self.cache, self.factors, self.k_new, self.v_new, self.err, stream)
 
     def route(self, scores=None, stream=None):
-        bk.route(self.cfg, self.cache, self.q, self.sel, self.sel_cnt, self.ws, self.err, scores, stream)
+        if self.routing == "head":
+            bk.route(self.cfg, self.cache, self.q, self.sel, self.sel_cnt, self.ws, self.err, scores, stream)
+        else:
+            bk.route_group(self.cfg, self.cache, self.q, _GROUP_REDUCE[self.routing], self.sel,
+                           self.sel_cnt, self.ws, self.err, scores, stream)
 
     def decode_attn(self, stream=None):
         bk.decode_attn(self.cfg, self.cache, self.q, self.sel, self.sel_cnt, self.o_lat, self.ws,

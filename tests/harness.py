@@ -37,7 +37,7 @@ class OracleCase:
         self.A, self.P, self.E = to64(case.A), to64(case.P), to64(case.E)
         self.G = O.fuse_out_factor(to64(case.Bf), to64(case.W_O), case.wl.num_q_heads, self.storage)
 
-    def sequence(self, b: int):
+    def sequence(self, b: int, routing: str = "head"):
         """Prefill all but the last token of sequence b, then one decode step."""
         wl = self.wl
         K = to64(self.case.keys[b])
@@ -45,7 +45,7 @@ class OracleCase:
         L = K.shape[0]
         cache = O.prefill(K[:-1], V[:-1], self.A, self.P, self.E, wl.page_size, self.storage, capacity=L)
         out = O.decode_step(cache, K[-1], V[-1], to64(self.case.q[b]), self.A, self.P, self.E,
-                            self.G, wl.top_k)
+                            self.G, wl.top_k, routing=routing)
         return cache, out
 
 

@@ -155,3 +155,20 @@ def test_noalloc_refuses_shapes_beyond_its_scratch(L):
     cache = bk.CCache(256, 256, 256, 256, 256, 256, 10, 4096)
     st = L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(cache), 256, 1024, 256, 256, 256, 256, None)
     assert st == bk.ERR_WORKSPACE
+
+
+def test_route_group_checks(L):
+    """basiskv_route_group: only GROUP_SUM / GROUP_MAX are reductions; the rest of its
+    validation is basiskv_route's (an empty batch launches nothing)."""
+    cfg = _cfg()
+    good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    for bad in (0, 3, -1):
+        assert L.basiskv_route_group(ctypes.byref(cfg), ctypes.byref(good), 256, 1, bad, 256, 256, None, 256,
+                                     1 << 30, 256, None) == bk.ERR_INVALID_ARG
+    for red in (bk.GROUP_SUM, bk.GROUP_MAX):
+        assert L.basiskv_route_group(ctypes.byref(cfg), ctypes.byref(good), 256, 0, red, 256, 256, None, None,
+                                     0, 256, None) == bk.OK
+        assert L.basiskv_route_group(ctypes.byref(cfg), None, 256, 1, red, 256, 256, None, 256, 1 << 30, 256,
+                                     None) == bk.ERR_INVALID_ARG
+        assert L.basiskv_route_group(ctypes.byref(cfg), ctypes.byref(good), 260, 1, red, 256, 256, None, 256,
+                                     1 << 30, 256, None) == bk.ERR_INVALID_ARG   # misaligned q

@@ -48,7 +48,7 @@ def _worker(rank, world, port, outdir):
         if r != 0:
             buf = io.StringIO()
             with contextlib.redirect_stdout(buf):
-                bench.run_reference(type("A", (), {"workload": "tiny_fp32", "warmup": 0, "steps": 1})(), w, r)
+                bench.run_reference(type("A", (), {"workload": "tiny_fp32", "warmup": 0, "steps": 1, "routing": "head"})(), w, r)
             res["ref_out"] = buf.getvalue()
         bench.barrier(w)
     finally:
