@@ -6,6 +6,8 @@
  *   basiskv_append       (step 1-2) store each new token's raw key, Value latent
  *                        and key residual in the paged cache; refresh the
  *                        summary (mean predicted key) of every page it touched
+ *                        (basiskv_prefill: the same for long appends, on the
+ *                        tensor cores)
  *   basiskv_route        (step 3)   score every page of every sequence for every
  *                        query head against the summaries; keep the top-k pages
  *                        plus the sink page and the recent page
@@ -159,6 +161,25 @@ BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basis
                               const basiskv_factors* factors, const void* k_new,
                               const void* v_new, int32_t batch, int32_t n_new,
                               int32_t* err_flag, void* stream);
+
+/*
+ * Steps 1-2 for long appends (prefill) on the tcgen05 tensor cores, bf16 only.
+ * Same arguments, layouts, results and error reporting as basiskv_append, with
+ * one difference in precision: the three chained products (C = v A_g,
+ * k - C P_g, R = (k - C P_g) E_g) accumulate in fp32 in tensor memory, and
+ * the fp32 intermediate that feeds the next product is passed as a bf16 pair
+ * (hi + lo, ~16 mantissa bits), so a stored C or R value may differ by one
+ * bf16 ulp from basiskv_append's correctly rounded fp64 result where the two
+ * straddle a rounding midpoint.  The summaries of every touched page are then
+ * recomputed in fp64 from the stored C and R, as basiskv_append does.
+ * Requires head_dim 64 or 128, rank_v a multiple of 16 in [16, 128], rank_k a
+ * multiple of 16 in [16, 64] (else BASISKV_ERR_UNSUPPORTED); k_new and v_new
+ * 16-byte aligned.  Worth it from a few hundred tokens per sequence on.
+ */
+BASISKV_API basiskv_status basiskv_prefill(const basiskv_config* cfg, const basiskv_cache* cache,
+                               const basiskv_factors* factors, const void* k_new,
+                               const void* v_new, int32_t batch, int32_t n_new,
+                               int32_t* err_flag, void* stream);
 
 /*
  * Step 3.  Page routing for every (sequence, query head).

@@ -26,7 +26,7 @@ DEVERR_BLOCK_TABLE, DEVERR_SELECTION, DEVERR_SEQ_LEN, DEVERR_TIMEOUT, DEVERR_WOR
 SYMBOLS = [
     "basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
     "basiskv_fuse_out_factor", "basiskv_workspace_bytes", "basiskv_status_string",
-    "basiskv_abi_version", "basiskv_decode_attn_noalloc", "basiskv_route_group",
+    "basiskv_abi_version", "basiskv_decode_attn_noalloc", "basiskv_route_group", "basiskv_prefill",
 ]
 
 
@@ -63,6 +63,7 @@ def lib():
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     pc, pk, pf = ctypes.POINTER(CConfig), ctypes.POINTER(CCache), ctypes.POINTER(CFactors)
     L.basiskv_append.argtypes = [pc, pk, pf, vp, vp, i32, i32, vp, vp]
+    L.basiskv_prefill.argtypes = [pc, pk, pf, vp, vp, i32, i32, vp, vp]
     L.basiskv_route.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, sz, vp, vp]
     L.basiskv_route_group.argtypes = [pc, pk, vp, i32, i32, vp, vp, vp, vp, sz, vp, vp]
     L.basiskv_decode_attn.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, sz, vp, vp]
@@ -76,7 +77,7 @@ def lib():
     L.basiskv_abi_version.argtypes = []
     for name in ["basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
                  "basiskv_fuse_out_factor", "basiskv_abi_version", "basiskv_decode_attn_noalloc",
-                 "basiskv_route_group"]:
+                 "basiskv_route_group", "basiskv_prefill"]:
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -205,6 +206,19 @@ def append(cfg: Config, cache: PagedCache, f: Factors, k_new: torch.Tensor, v_ne
     _check(lib().basiskv_append(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), ctypes.byref(f.c()),
                                 _ptr(k_new), _ptr(v_new), B, n_new, _ptr(err), _stream(stream)),
            "basiskv_append")
+
+
+def prefill(cfg: Config, cache: PagedCache, f: Factors, k_new: torch.Tensor, v_new: torch.Tensor,
+            err: torch.Tensor, stream=None):
+    """basiskv_append for long appends on the tensor cores (bf16): k_new, v_new [B, n_new, Hkv, d]."""
+    B, n_new = k_new.shape[0], k_new.shape[1]
+    shape = (B, n_new, cfg.num_kv_heads, cfg.head_dim)
+    _need(k_new, "k_new", cfg.dtype, shape)
+    _need(v_new, "v_new", cfg.dtype, shape)
+    _need(err, "err", torch.int32)
+    _check(lib().basiskv_prefill(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), ctypes.byref(f.c()),
+                                 _ptr(k_new), _ptr(v_new), B, n_new, _ptr(err), _stream(stream)),
+           "basiskv_prefill")
 
 
 def route(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor, sel_cnt: torch.Tensor,

@@ -125,6 +125,27 @@ basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* ca
   return cuda_status(launch_append(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
 }
 
+basiskv_status basiskv_prefill(const basiskv_config* cfg, const basiskv_cache* cache,
+                               const basiskv_factors* f, const void* k_new, const void* v_new,
+                               int32_t batch, int32_t n_new, int32_t* err_flag, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != BASISKV_OK) return s;
+  if (!prefill_tc_supported(cfg->dtype == BASISKV_BF16, cfg->head_dim, cfg->rank_v, cfg->rank_k))
+    return BASISKV_ERR_UNSUPPORTED;
+  if (batch == 0 || n_new == 0) return BASISKV_OK;
+  if (!f || !f->A || !f->P || !f->E || !k_new || !v_new || !err_flag || batch < 0 || n_new < 0)
+    return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(f->A) || !aligned16(f->P) || !aligned16(f->E) || !aligned16(k_new) || !aligned16(v_new))
+    return BASISKV_ERR_INVALID_ARG;
+  if ((long long)n_new > (long long)cache->max_pages * cfg->page_size) return BASISKV_ERR_INVALID_ARG;
+  const AppendParams p{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
+                       cache->summary, cache->block_table, cache->seq_len, err_flag,
+                       batch, n_new, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
+                       cfg->page_size, cache->max_pages, cache->num_phys_pages, nullptr, 0};
+  return cuda_status(launch_prefill_tc(p, num_sms(), (cudaStream_t)stream));
+}
+
 static basiskv_status route_common(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
                                    int32_t batch, int group_mode, int32_t* sel, int32_t* sel_cnt, float* scores,
                                    void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {

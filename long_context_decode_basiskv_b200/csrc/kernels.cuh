@@ -23,6 +23,9 @@ struct AppendParams {
   size_t warm_bytes;  // a multiple of 16
 };
 cudaError_t launch_append(const AppendParams& p, bool bf16, cudaStream_t st);
+// many tokens per sequence on the tensor cores (bf16 only), then the touched pages' summaries
+bool prefill_tc_supported(bool bf16, int d, int r, int s);
+cudaError_t launch_prefill_tc(const AppendParams& p, int num_sms, cudaStream_t st);
 
 struct RouteParams {
   const void* q;

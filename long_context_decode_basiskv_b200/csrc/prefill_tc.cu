@@ -1,0 +1,411 @@
+// Steps 1-2 for many tokens at once (prefill): the latent and residual of
+// every new token on the tcgen05 tensor cores, then the summaries of every
+// page the tokens touched.
+//
+// Per token and KV head g (BasisKV abstract; kongchang.com explainer, section
+// "用Value潜变量辅助Key路由"):  C = v A_g,  R = (k - C P_g) E_g  with R from
+// the unrounded C.  For a tile of 128 tokens of one (sequence, KV head) these
+// are three chained matrix products, M = 128 tokens each:
+//
+//   MMA 1   C [128 x r]  = V [128 x d] . A_g              (K = d)
+//   MMA 2   X [128 x d]  = C . P_g                        (K = r)
+//   MMA 3   R [128 x s]  = (K - X) [128 x d] . E_g        (K = d)
+//
+// with bf16 operands in shared memory and fp32 accumulators in tensor memory.
+// The fp32 results of MMA 1 and of K - X are fed to the next product as two
+// bf16 operands, hi = bf16(x) and lo = bf16(x - hi), multiplied into the same
+// accumulator: the chained operand keeps ~16 bits of mantissa instead of 8,
+// so R is formed from C at nearly fp32 precision (the unrounded C the method
+// asks for), not from the stored bf16 C.
+//
+// One CTA of 128 threads per (sequence, KV head, share of the tiles); thread 0
+// issues the MMAs, each of the 4 warps reads its 32 accumulator lanes (= 32
+// tokens) back with tcgen05.ld.  The factors are staged once per CTA,
+// transposed into the K-major swizzled operand layout.  Stored values: the raw
+// key, C and R rounded once to bf16 (fp32 accumulation: a value can differ by
+// one bf16 ulp from the correctly rounded fp64 result where the two straddle a
+// rounding midpoint).
+//
+// The page summaries S = mean(C) P_g + mean(R) E_g^T over each touched page's
+// valid tokens (old and new) are recomputed afterwards by a second kernel, in
+// fp64 from the stored C and R, one CTA per (sequence, KV head, 32 pages) with
+// the factors staged once.
+#include "kernels.cuh"
+#include "tcgen05.cuh"
+
+namespace bkv {
+
+constexpr int kPfM = 128;          // tokens per tile (the MMA's M)
+constexpr int kPfThreads = 128;    // 4 warps: one per 32 accumulator lanes
+constexpr uint32_t kAtom = 16384;  // one 128-row x 128-byte swizzle atom column of an M = 128 operand
+
+// byte offset of element (row, k) of a K-major, 128-byte-swizzled bf16 operand
+// with `rows` rows: atoms of 64 K-elements are rows * 128 bytes apart
+__device__ __forceinline__ uint32_t sw_off(int row, int k, int rows) {
+  const int atom = k >> 6, kk = k & 63;
+  return (uint32_t)atom * (uint32_t)rows * 128u + (uint32_t)row * 128u +
+         ((uint32_t)((kk >> 3) ^ (row & 7)) << 4) + (uint32_t)(kk & 7) * 2u;
+}
+
+// descriptor of K-step j (16 elements) of a K-major swizzled operand with `rows` rows
+__device__ __forceinline__ uint64_t kstep_desc(const unsigned char* base, int j, int rows) {
+  return smem_desc_sw128(base + (size_t)(j >> 2) * rows * 128) + (uint64_t)((j & 3) * 32 >> 4);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
+}
+
+// hi/lo split of 8 fp32 values into two 16-byte bf16 chunks
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float a = x[2 * j], b = x[2 * j + 1];
+    const float ah = __bfloat162float(__float2bfloat16_rn(a)), bh = __bfloat162float(__float2bfloat16_rn(b));
+    h[j] = pack_bf16(ah, bh);
+    l[j] = pack_bf16(a - ah, b - bh);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+struct PfLayout {
+  uint32_t b1, b2, b3, v, k, chi, clo, bar, slot, total;
+};
+
+__host__ __device__ inline int pf_atoms(int kdim) { return (kdim + 63) / 64; }
+
+__host__ __device__ inline PfLayout pf_layout(int d, int r, int s) {
+  PfLayout L{};
+  uint32_t o = 0;
+  L.b1 = o;  o += (uint32_t)pf_atoms(d) * r * 128;  // A_g^T: r rows, K = d
+  L.b2 = o;  o += (uint32_t)pf_atoms(r) * d * 128;  // P_g^T: d rows, K = r
+  L.b3 = o;  o += (uint32_t)pf_atoms(d) * s * 128;  // E_g^T: s rows, K = d
+  L.v = o;   o += (uint32_t)pf_atoms(d) * kAtom;    // V tile, then (K - X) hi
+  L.k = o;   o += (uint32_t)pf_atoms(d) * kAtom;    // K tile, then (K - X) lo
+  L.chi = o; o += (uint32_t)pf_atoms(r) * kAtom;    // C hi
+  L.clo = o; o += (uint32_t)pf_atoms(r) * kAtom;    // C lo
+  L.bar = o; o += 16;
+  L.slot = o; o += 16;
+  L.total = o;
+  return L;
+}
+
+__host__ __device__ inline uint32_t pf_tmem_cols(int d, int r, int s) {
+  const int need = ((r + 31) / 32) * 32 + ((d + 31) / 32) * 32 + ((s + 31) / 32) * 32;
+  uint32_t c = 32;
+  while ((int)c < need) c <<= 1;
+  return c;
+}
+
+__global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int d = p.d, r = p.r, s = p.s, P = p.page;
+  const int L = p.seq_len[b];
+  if (L < p.n_new || L > p.max_pages * P || p.n_new <= 0) {
+    if (tid == 0 && blockIdx.x == 0) set_err(p.err, BASISKV_DEVERR_SEQ_LEN);
+    return;
+  }
+  const int first = L - p.n_new;
+  const int ntiles = (p.n_new + kPfM - 1) / kPfM;
+  if ((int)blockIdx.x >= ntiles) return;
+
+  const PfLayout lay = pf_layout(d, r, s);
+  unsigned char* sB1 = smem + lay.b1;
+  unsigned char* sB2 = smem + lay.b2;
+  unsigned char* sB3 = smem + lay.b3;
+  unsigned char* sV = smem + lay.v;
+  unsigned char* sK = smem + lay.k;
+  unsigned char* sChi = smem + lay.chi;
+  unsigned char* sClo = smem + lay.clo;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + lay.bar);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + lay.slot);
+  __shared__ int s_fail;
+
+  const uint32_t ncols = pf_tmem_cols(d, r, s);
+  const uint32_t colC = 0, colX = (uint32_t)((r + 31) / 32) * 32, colR = colX + (uint32_t)((d + 31) / 32) * 32;
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      s_fail = 0;
+    }
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+
+  // factors of head g, transposed into the K-major operand layout (N rows, K contiguous)
+  const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(p.A) + (size_t)g * d * r;  // [d][r]
+  const __nv_bfloat16* Pm = static_cast<const __nv_bfloat16*>(p.P) + (size_t)g * r * d; // [r][d]
+  const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(p.E) + (size_t)g * d * s;  // [d][s]
+  // zero the unused K tail of the P^T atoms (r not a multiple of 64)
+  for (int i = tid; i < pf_atoms(r) * d * 8; i += kPfThreads)
+    reinterpret_cast<uint4*>(sB2)[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < pf_atoms(r) * (int)(kAtom / 16); i += kPfThreads) {
+    reinterpret_cast<uint4*>(sChi)[i] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(sClo)[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+  for (int i = tid; i < d * r; i += kPfThreads) {  // A^T[j][x] = A[x][j]
+    const int x = i / r, j = i - x * r;
+    *reinterpret_cast<__nv_bfloat16*>(sB1 + sw_off(j, x, r)) = A[i];
+  }
+  for (int i = tid; i < r * d; i += kPfThreads) {  // P^T[x][j] = P[j][x]
+    const int j = i / d, x = i - j * d;
+    *reinterpret_cast<__nv_bfloat16*>(sB2 + sw_off(x, j, d)) = Pm[i];
+  }
+  for (int i = tid; i < d * s; i += kPfThreads) {  // E^T[q][x] = E[x][q]
+    const int x = i / s, q = i - x * s;
+    *reinterpret_cast<__nv_bfloat16*>(sB3 + sw_off(q, x, s)) = E[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t lanes = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
+
+  const bool swz_on = kc_swizzled(true, d, r);
+  const int mk = swz_on ? swz_mask(d) : 0, mc = swz_on ? swz_mask(r) : 0;
+  const __nv_bfloat16* kin = static_cast<const __nv_bfloat16*>(p.k_new);
+  const __nv_bfloat16* vin = static_cast<const __nv_bfloat16*>(p.v_new);
+  __nv_bfloat16* kraw = static_cast<__nv_bfloat16*>(p.k_raw);
+  __nv_bfloat16* clat = static_cast<__nv_bfloat16*>(p.c_lat);
+  __nv_bfloat16* rres = static_cast<__nv_bfloat16*>(p.r_res);
+  const int cpr = d / 8;  // 16-byte chunks per k / v row
+  const uint32_t id1 = idesc_bf16(kPfM, r), id2 = idesc_bf16(kPfM, d), id3 = idesc_bf16(kPfM, s);
+  uint32_t phase = 0;
+  bool ok = true;
+
+  // cache block of token `tok` of this tile's sequence (-1: invalid page, skipped)
+  auto token_block = [&](int tok, int& slot) -> long long {
+    const int pos = first + tok;
+    const int page = pos / P;
+    slot = pos - page * P;
+    const int phys = p.block_table[(size_t)b * p.max_pages + page];
+    if (phys < 0 || phys >= p.num_phys) {
+      set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
+      return -1;
+    }
+    return (long long)phys * p.Hkv + g;
+  };
+  auto wait_mma = [&]() {
+    if (tid == 0) s_fail |= mbar_wait_bounded(bar, phase) ? 0 : 1;
+    phase ^= 1u;
+    __syncthreads();
+    tc_fence_after();
+    if (s_fail) ok = false;
+  };
+
+  for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+    const int t0 = tile * kPfM;
+    // k and v rows of the tile -> swizzled operand tiles; raw keys -> the cache
+    for (int q = tid; q < kPfM * cpr; q += kPfThreads) {
+      const int row = q / cpr, c = q - row * cpr;
+      const int tok = t0 + row;
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+      if (tok < p.n_new) {
+        const size_t src = (((size_t)b * p.n_new + tok) * p.Hkv + g) * d + (size_t)c * 8;
+        kv = __ldg(reinterpret_cast<const uint4*>(kin + src));
+        vv = __ldg(reinterpret_cast<const uint4*>(vin + src));
+        int slot;
+        const long long blk = token_block(tok, slot);
+        if (blk >= 0)
+          *reinterpret_cast<uint4*>(kraw + ((size_t)blk * P + slot) * d + (size_t)((c ^ (slot & mk)) * 8)) = kv;
+      }
+      const uint32_t off = sw_off(row, c * 8, kPfM);
+      *reinterpret_cast<uint4*>(sV + off) = vv;
+      *reinterpret_cast<uint4*>(sK + off) = kv;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      for (int j = 0; j < d / 16; ++j)
+        tc_mma(tmem + colC, kstep_desc(sV, j, kPfM), kstep_desc(sB1, j, r), id1, j > 0 ? 1u : 0u);
+      tc_commit(bar);
+    }
+    wait_mma();
+    if (!ok) break;
+
+    // C: this thread's token row -> stored C (bf16) and the hi / lo operand of MMA 2
+    const int row = warp * 32 + lane;
+    const int tok = t0 + row;
+    int slot = 0;
+    const long long blk = (tok < p.n_new) ? token_block(tok, slot) : -1;
+    for (int c0 = 0; c0 < r; c0 += 16) {
+      float v[16];
+      tc_ld16(tmem + lanes + colC + (uint32_t)c0, v);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint4 hi, lo;
+        split8(v + 8 * h, hi, lo);
+        const int k = c0 + 8 * h;
+        *reinterpret_cast<uint4*>(sChi + sw_off(row, k, kPfM)) = hi;
+        *reinterpret_cast<uint4*>(sClo + sw_off(row, k, kPfM)) = lo;
+        if (blk >= 0)
+          *reinterpret_cast<uint4*>(clat + ((size_t)blk * P + slot) * r + (size_t)(((k >> 3) ^ (slot & mc)) * 8)) = hi;
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      for (int j = 0; j < r / 16; ++j)
+        tc_mma(tmem + colX, kstep_desc(sChi, j, kPfM), kstep_desc(sB2, j, d), id2, j > 0 ? 1u : 0u);
+      for (int j = 0; j < r / 16; ++j)
+        tc_mma(tmem + colX, kstep_desc(sClo, j, kPfM), kstep_desc(sB2, j, d), id2, 1u);
+      tc_commit(bar);
+    }
+    wait_mma();
+    if (!ok) break;
+
+    // U = k - X: hi into the V tile, lo over the K tile (each row is this thread's own)
+    for (int c0 = 0; c0 < d; c0 += 16) {
+      float x[16];
+      tc_ld16(tmem + lanes + colX + (uint32_t)c0, x);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int k = c0 + 8 * h;
+        const uint32_t off = sw_off(row, k, kPfM);
+        const uint4 kq = *reinterpret_cast<const uint4*>(sK + off);
+        const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w};
+        float u[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          u[2 * e] = bf16lo(kw[e]) - x[8 * h + 2 * e];
+          u[2 * e + 1] = bf16hi(kw[e]) - x[8 * h + 2 * e + 1];
+        }
+        uint4 hi, lo;
+        split8(u, hi, lo);
+        *reinterpret_cast<uint4*>(sV + off) = hi;
+        *reinterpret_cast<uint4*>(sK + off) = lo;
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      for (int j = 0; j < d / 16; ++j)
+        tc_mma(tmem + colR, kstep_desc(sV, j, kPfM), kstep_desc(sB3, j, s), id3, j > 0 ? 1u : 0u);
+      for (int j = 0; j < d / 16; ++j)
+        tc_mma(tmem + colR, kstep_desc(sK, j, kPfM), kstep_desc(sB3, j, s), id3, 1u);
+      tc_commit(bar);
+    }
+    wait_mma();
+    if (!ok) break;
+
+    // R -> the cache (rows not swizzled)
+    for (int c0 = 0; c0 < s; c0 += 16) {
+      float v[16];
+      tc_ld16(tmem + lanes + colR + (uint32_t)c0, v);
+      if (blk >= 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 o = make_uint4(pack_bf16(v[8 * h], v[8 * h + 1]), pack_bf16(v[8 * h + 2], v[8 * h + 3]),
+                                     pack_bf16(v[8 * h + 4], v[8 * h + 5]), pack_bf16(v[8 * h + 6], v[8 * h + 7]));
+          *reinterpret_cast<uint4*>(rres + ((size_t)blk * P + slot) * s + c0 + 8 * h) = o;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // smem tiles and TMEM are reused by the next tile
+    tc_fence_after();
+  }
+  if (!ok && tid == 0) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// page summaries of every page the appended tokens touched
+// ---------------------------------------------------------------------------
+constexpr int kSumPages = 32;  // pages per CTA
+constexpr int kSumThreads = 128;
+
+__global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int b = blockIdx.z, g = blockIdx.y, tid = threadIdx.x;
+  const int d = p.d, r = p.r, s = p.s, P = p.page;
+  const int L = p.seq_len[b];
+  if (L < p.n_new || L > p.max_pages * P || p.n_new <= 0) return;  // reported by the latent kernel
+  const int first_page = (L - p.n_new) / P;
+  const int last_page = (L - 1) / P;
+  const int pg0 = first_page + blockIdx.x * kSumPages;
+  if (pg0 > last_page) return;
+  float* sP = reinterpret_cast<float*>(smem);  // [r][d]
+  float* sE = sP + r * d;                      // [d][s]
+  double* sMean = reinterpret_cast<double*>(sE + d * s);  // [r + s]
+  const __nv_bfloat16* Pm = static_cast<const __nv_bfloat16*>(p.P) + (size_t)g * r * d;
+  const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(p.E) + (size_t)g * d * s;
+  for (int i = tid; i < r * d; i += kSumThreads) sP[i] = __bfloat162float(Pm[i]);
+  for (int i = tid; i < d * s; i += kSumThreads) sE[i] = __bfloat162float(E[i]);
+  const bool swz_on = kc_swizzled(true, d, r);
+  const int mc = swz_on ? swz_mask(r) : 0;
+  const __nv_bfloat16* clat = static_cast<const __nv_bfloat16*>(p.c_lat);
+  const __nv_bfloat16* rres = static_cast<const __nv_bfloat16*>(p.r_res);
+  for (int page = pg0; page <= min(last_page, pg0 + kSumPages - 1); ++page) {
+    const int phys = p.block_table[(size_t)b * p.max_pages + page];
+    __syncthreads();  // factors staged / the previous page's sMean consumed
+    if (phys < 0 || phys >= p.num_phys) continue;  // reported by the latent kernel
+    const size_t blk = (size_t)phys * p.Hkv + g;
+    const int m = min(L, (page + 1) * P) - page * P;
+    for (int j = tid; j < r + s; j += kSumThreads) {
+      double acc = 0.0;
+      if (j < r) {
+        for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(clat[(blk * P + t) * r + swz(j, t, mc)]);
+      } else {
+        for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(rres[(blk * P + t) * s + (j - r)]);
+      }
+      sMean[j] = acc / (double)m;
+    }
+    __syncthreads();
+    for (int x = tid; x < d; x += kSumThreads) {
+      double acc = 0.0;
+      for (int j = 0; j < r; ++j) acc = fma(sMean[j], (double)sP[j * d + x], acc);
+      double acc2 = 0.0;
+      for (int q = 0; q < s; ++q) acc2 = fma(sMean[r + q], (double)sE[x * s + q], acc2);
+      p.summary[blk * d + x] = __double2float_rn(acc + acc2);
+    }
+  }
+}
+
+bool prefill_tc_supported(bool bf16, int d, int r, int s) {
+  return bf16 && (d == 64 || d == 128) && r >= 16 && r <= 128 && r % 16 == 0 && s >= 16 && s <= 64 &&
+         s % 16 == 0 && pf_layout(d, r, s).total + 1024 <= 227 * 1024;
+}
+
+cudaError_t launch_prefill_tc(const AppendParams& p, int num_sms, cudaStream_t st) {
+  const PfLayout lay = pf_layout(p.d, p.r, p.s);
+  const size_t smem = lay.total + 1024;  // + alignment of the dynamic window to 1024 bytes
+  cudaError_t e = ensure_smem((const void*)prefill_tc_kernel, smem);
+  if (e != cudaSuccess) return e;
+  const int ntiles = (p.n_new + kPfM - 1) / kPfM;
+  const int groups = p.batch * p.Hkv;
+  const int split = std::max(1, std::min(ntiles, num_sms / std::max(1, groups)));
+  prefill_tc_kernel<<<dim3(split, p.Hkv, p.batch), kPfThreads, smem, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t ssmem = (size_t)(p.r * p.d + p.d * p.s) * sizeof(float) + (size_t)(p.r + p.s) * sizeof(double);
+  if ((e = ensure_smem((const void*)page_summary_kernel, ssmem)) != cudaSuccess) return e;
+  // pages touched by n_new tokens starting anywhere inside a page
+  const int touched = (p.n_new + p.page - 1) / p.page + 1;
+  page_summary_kernel<<<dim3((touched + kSumPages - 1) / kSumPages, p.Hkv, p.batch), kSumThreads, ssmem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace bkv

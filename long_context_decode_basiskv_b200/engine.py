@@ -6,7 +6,9 @@ out-projection factor (built by the library's fusion kernel), the step's
 inputs and outputs, and one workspace.  ``step()`` enqueues the four calls of
 one decode step: append, route, decode_attn, out_proj.  ``routing`` picks one
 selection per query head ("head") or per KV group from the sum ("group_sum")
-or maximum ("group_max") of its heads' page scores.
+or maximum ("group_max") of its heads' page scores.  ``prefill_mode`` builds
+the cache with basiskv_append ("exact", fp64 sums) or basiskv_prefill ("tc",
+the tensor-core path for long appends).
 """
 from __future__ import annotations
 
@@ -26,10 +28,14 @@ _GROUP_REDUCE = {"group_sum": bk.GROUP_SUM, "group_max": bk.GROUP_MAX}
 
 
 class DecodeEngine:
-    def __init__(self, case: Case, device="cuda", stream=None, routing: str = "head"):
+    def __init__(self, case: Case, device="cuda", stream=None, routing: str = "head",
+                 prefill_mode: str = "exact"):
         if routing != "head" and routing not in _GROUP_REDUCE:
             raise ValueError(f"routing must be 'head', 'group_sum' or 'group_max', not {routing!r}")
+        if prefill_mode not in ("exact", "tc"):
+            raise ValueError(f"prefill_mode must be 'exact' or 'tc', not {prefill_mode!r}")
         self.routing = routing
+        self.prefill_mode = prefill_mode
         self.case = case
         self.cfg = cfg = config_of(case)
         self.device = torch.device(device)
@@ -85,7 +91,8 @@ class DecodeEngine:
             sub.seq_len = torch.tensor([L - 1], dtype=torch.int32, device=dev)
             k = case.keys[b][:-1].to(dev).unsqueeze(0).contiguous()
             v = case.values[b][:-1].to(dev).unsqueeze(0).contiguous()
-            bk.append(cfg, sub, self.factors, k, v, self.err, stream)
+            fn = bk.prefill if self.prefill_mode == "tc" else bk.append
+            fn(cfg, sub, self.factors, k, v, self.err, stream)
 
     def append(self, stream=None):
         bk.append(self.cfg, self.cache, self.factors, self.k_new, self.v_new, self.err, stream)

@@ -172,3 +172,22 @@ def test_route_group_checks(L):
                                      None) == bk.ERR_INVALID_ARG
         assert L.basiskv_route_group(ctypes.byref(cfg), ctypes.byref(good), 260, 1, red, 256, 256, None, 256,
                                      1 << 30, 256, None) == bk.ERR_INVALID_ARG   # misaligned q
+
+
+def test_prefill_checks(L):
+    """basiskv_prefill: bf16 with ranks that are multiples of 16 only; otherwise basiskv_append's checks."""
+    good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    f = bk.CFactors(256, 256, 256, 256)
+    for bad in (dict(dtype=bk.F32), dict(rank_k=8), dict(rank_v=24), dict(head_dim=96, rank_v=32)):
+        cfg = _cfg(**bad)
+        assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 1, 64, 256,
+                                 None) == bk.ERR_UNSUPPORTED, bad
+    cfg = _cfg()
+    assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 0, 64, 256,
+                             None) == bk.OK
+    assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 264, 256, 1, 64, 256,
+                             None) == bk.ERR_INVALID_ARG                       # misaligned k_new
+    assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 1, 64, None,
+                             None) == bk.ERR_INVALID_ARG                       # no error flag
+    assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 1, 161, 256,
+                             None) == bk.ERR_INVALID_ARG                       # more tokens than the block table holds
