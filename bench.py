@@ -62,6 +62,7 @@ def parse():
                     help="decode steps per sampled sequence in the CPU baseline (about 10 s in total)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-append measurement")
     return ap.parse_args()
 
 
@@ -256,6 +257,55 @@ def oracle_sample(case, nseq: int, repeats: int = 1, routing: str = "head"):
 
 
 # ---------------------------------------------------------------------------
+# prefill append: the whole context of every sequence in one call
+# ---------------------------------------------------------------------------
+def measure_prefill(eng, stream, reps: int = 3):
+    """Time basiskv_prefill (tensor cores) and basiskv_append (fp64) rebuilding the
+    cache of all but the last token of every sequence (equal lengths only: one
+    call for the batch).  Runs after the decode measurements; it rewrites the
+    cache with the tensor-core values.  Returns a dict, or None for ragged batches."""
+    from long_context_decode_basiskv_b200 import binding as bk
+
+    case, cfg = eng.case, eng.cfg
+    lengths = set(case.lengths)
+    if len(lengths) != 1 or cfg.dtype != torch.bfloat16:
+        return None
+    L = lengths.pop()
+    B = case.wl.batch
+    k = torch.stack([x[:-1] for x in case.keys]).contiguous()
+    v = torch.stack([x[:-1] for x in case.values]).contiguous()
+    sub = bk.PagedCache.__new__(bk.PagedCache)
+    sub.__dict__.update(eng.cache.__dict__)
+    sub.seq_len = torch.full((B,), L - 1, dtype=torch.int32, device=k.device)
+    res = {"tokens": B * (L - 1)}
+    with torch.cuda.stream(stream):
+        for name, fn in [("tensor_core", bk.prefill), ("fp64_append", bk.append)]:
+            fn(cfg, sub, eng.factors, k, v, eng.err)  # warm-up
+            evs = []
+            for _ in range(reps):
+                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn(cfg, sub, eng.factors, k, v, eng.err)
+                b_.record(stream)
+                evs.append((a, b_))
+            torch.cuda.synchronize()
+            us = sum(a.elapsed_time(b_) for a, b_ in evs) / reps * 1e3
+            res[name] = {"us": round(us, 1), "tokens_per_s": round(B * (L - 1) / (us * 1e-6), 1)}
+    # bytes the tensor-core path must move: k, v in; raw k, C, R out; C, R re-read for the
+    # summaries; one fp32 summary row per page and head
+    d, r, s_, P = cfg.head_dim, cfg.rank_v, cfg.rank_k, cfg.page_size
+    tok_heads = B * (L - 1) * cfg.num_kv_heads
+    nbytes = tok_heads * (3 * d * 2 + 2 * (r + s_) * 2) + B * (-(-(L - 1) // P)) * cfg.num_kv_heads * d * 4
+    peak, kind = measured_peak()
+    gbs = nbytes / (res["tensor_core"]["us"] * 1e-6) / 1e9
+    res["roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                       "frac": round(gbs / peak, 4), "algorithmic_bytes": nbytes,
+                       "peak_source": f"{kind} copy bandwidth"}
+    res["err"] = int(eng.err.item())
+    return res
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def run_ours(args, world, rank, local):
@@ -371,6 +421,10 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                "ms_per_step": round(e2e_ms / args.steps, 4)}
 
+    prefill = None
+    if not args.no_prefill:
+        prefill = measure_prefill(eng, stream)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         times, desc = oracle_sample(case, args.oracle_seqs, args.oracle_repeats, args.routing)
@@ -400,6 +454,7 @@ def run_ours(args, world, rank, local):
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
             "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -207,23 +207,30 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
 
   for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
     const int t0 = tile * kPfM;
-    // k and v rows of the tile -> swizzled operand tiles; raw keys -> the cache
-    for (int q = tid; q < kPfM * cpr; q += kPfThreads) {
-      const int row = q / cpr, c = q - row * cpr;
-      const int tok = t0 + row;
-      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
-      if (tok < p.n_new) {
-        const size_t src = (((size_t)b * p.n_new + tok) * p.Hkv + g) * d + (size_t)c * 8;
-        kv = __ldg(reinterpret_cast<const uint4*>(kin + src));
-        vv = __ldg(reinterpret_cast<const uint4*>(vin + src));
-        int slot;
-        const long long blk = token_block(tok, slot);
-        if (blk >= 0)
-          *reinterpret_cast<uint4*>(kraw + ((size_t)blk * P + slot) * d + (size_t)((c ^ (slot & mk)) * 8)) = kv;
+    // k and v rows of the tile -> swizzled operand tiles, 8 chunks of each in flight per thread
+    for (int i0 = 0; i0 < kPfM * cpr / kPfThreads; i0 += 8) {
+      uint4 kq[8], vq[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = tid + kPfThreads * (i0 + u);
+        const int row = q / cpr, c = q - row * cpr;
+        const int tok = t0 + row;
+        kq[u] = make_uint4(0u, 0u, 0u, 0u);
+        vq[u] = kq[u];
+        if (tok < p.n_new) {
+          const size_t src = (((size_t)b * p.n_new + tok) * p.Hkv + g) * d + (size_t)c * 8;
+          kq[u] = __ldg(reinterpret_cast<const uint4*>(kin + src));
+          vq[u] = __ldg(reinterpret_cast<const uint4*>(vin + src));
+        }
       }
-      const uint32_t off = sw_off(row, c * 8, kPfM);
-      *reinterpret_cast<uint4*>(sV + off) = vv;
-      *reinterpret_cast<uint4*>(sK + off) = kv;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = tid + kPfThreads * (i0 + u);
+        const int row = q / cpr, c = q - row * cpr;
+        const uint32_t off = sw_off(row, c * 8, kPfM);
+        *reinterpret_cast<uint4*>(sV + off) = vq[u];
+        *reinterpret_cast<uint4*>(sK + off) = kq[u];
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -237,11 +244,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
     wait_mma();
     if (!ok) break;
 
-    // C: this thread's token row -> stored C (bf16) and the hi / lo operand of MMA 2
+    // this thread's token row: the raw key from the K tile -> the cache
     const int row = warp * 32 + lane;
     const int tok = t0 + row;
     int slot = 0;
     const long long blk = (tok < p.n_new) ? token_block(tok, slot) : -1;
+    if (blk >= 0) {
+      for (int c = 0; c < cpr; ++c)
+        *reinterpret_cast<uint4*>(kraw + ((size_t)blk * P + slot) * d + (size_t)((c ^ (slot & mk)) * 8)) =
+            *reinterpret_cast<const uint4*>(sK + sw_off(row, c * 8, kPfM));
+    }
+    // C -> stored C (bf16) and the hi / lo operand of MMA 2
     for (int c0 = 0; c0 < r; c0 += 16) {
       float v[16];
       tc_ld16(tmem + lanes + colC + (uint32_t)c0, v);
