@@ -60,7 +60,9 @@
 extern "C" {
 #endif
 
-#define BASISKV_ABI_VERSION 1
+/* 1: append, route, decode_attn, out_proj and their helpers;
+ * 2: adds basiskv_route_group and basiskv_prefill (nothing earlier changed). */
+#define BASISKV_ABI_VERSION 2
 
 typedef enum {
   BASISKV_OK = 0,
