@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-append measurement")
+    ap.add_argument("--tp", action="store_true",
+                    help="shard the heads of one workload over the N ranks (one NCCL all-reduce of y per "
+                         "step) instead of running N independent replicas")
     return ap.parse_args()
 
 
@@ -314,8 +317,21 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_dist(world, "nccl")
-    wl = replica_workload(WORKLOADS[args.workload], rank, world)
-    case = make_case(wl, dev)
+    if args.tp:
+        from long_context_decode_basiskv_b200.tensor_parallel import reduce_y, shard_case
+
+        full_wl = WORKLOADS[args.workload]
+        case = shard_case(make_case(full_wl, dev), rank, world)   # every rank builds the same case
+        wl = case.wl
+        tokens_per_step = full_wl.batch                           # the ranks share one batch
+    else:
+        full_wl = wl = replica_workload(WORKLOADS[args.workload], rank, world)
+        case = make_case(wl, dev)
+        tokens_per_step = world * wl.batch                        # independent replicas
+
+    def exchange():
+        if args.tp:
+            reduce_y(eng.y, world)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         eng = DecodeEngine(case, device=dev, routing=args.routing)
@@ -348,6 +364,8 @@ def run_ours(args, world, rank, local):
                     e[0].record(stream)
                 for i, name in enumerate(phases):
                     graphs[name].replay()
+                    if name == "step":
+                        exchange()
                     if record:
                         e[i + 1].record(stream)
                 if record:
@@ -370,7 +388,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, name in enumerate(order)}
     ms_per_step = total_ms / args.steps
-    value = world * wl.batch * args.steps / (total_ms / 1e3)
+    value = tokens_per_step * args.steps / (total_ms / 1e3)
 
     mean = {k: sum(v) / len(v) for k, v in per.items()}
     peak, peak_kind = measured_peak()
@@ -404,6 +422,7 @@ def run_ours(args, world, rank, local):
                         a.record(stream)
                     eng.input_buffer().copy_(hin, non_blocking=True)
                     eng.graph_step()
+                    exchange()
                     hy.copy_(eng.y, non_blocking=True)
                     if record:
                         b_.record(stream)
@@ -417,7 +436,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in pairs), world, dev)
-        e2e = {"value": round(world * wl.batch * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+        e2e = {"value": round(tokens_per_step * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
                "ms_per_step": round(e2e_ms / args.steps, 4)}
 
@@ -435,13 +454,15 @@ def run_ours(args, world, rank, local):
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if args.tp else "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic (seeded generator)",
-            "config": {"workload": wl.name, "batch": wl.batch, "context": wl.context if not wl.ragged else list(wl.ragged),
-                       "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+            "config": {"workload": full_wl.name, "batch": full_wl.batch,
+                       "context": full_wl.context if not full_wl.ragged else list(full_wl.ragged),
+                       "q_heads": full_wl.num_q_heads, "kv_heads": full_wl.num_kv_heads, "head_dim": wl.head_dim,
                        "page_size": wl.page_size, "rank_v": wl.rank_v, "rank_k": wl.rank_k,
                        "top_k": wl.top_k, "hidden": wl.hidden, "routing": args.routing,
-                       "parallelism": f"replicas x{world}",
+                       "parallelism": (f"tp{world}: KV heads sharded, NCCL all-reduce of y per step"
+                                       if args.tp else f"replicas x{world}"),
                        "l2": "flushed between steps (read of a 256 MiB buffer)",
                        "timing": "one CUDA graph per step (append || route on forked streams, decode_attn, out_proj), CUDA events around each replay; kernels_us from per-phase graphs in a separate pass; route+attn GB/s counts the append || route phase time"},
             "kernels_us": {k: round(v * 1e3, 2) for k, v in mean.items()},
