@@ -176,7 +176,8 @@ BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basis
  * recomputed in fp64 from the stored C and R, as basiskv_append does.
  * Requires head_dim 64 or 128, rank_v a multiple of 16 in [16, 128], rank_k a
  * multiple of 16 in [16, 64] (else BASISKV_ERR_UNSUPPORTED); k_new and v_new
- * 16-byte aligned.  Worth it from a few hundred tokens per sequence on.
+ * 16-byte aligned.  Work is split in tiles of 128 consecutive new tokens per
+ * (sequence, KV head), so short appends leave most of the GPU idle.
  */
 BASISKV_API basiskv_status basiskv_prefill(const basiskv_config* cfg, const basiskv_cache* cache,
                                const basiskv_factors* factors, const void* k_new,
