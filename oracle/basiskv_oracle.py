@@ -51,7 +51,7 @@ import numpy as np
 __all__ = [
     "round_storage", "append_latents", "page_summaries", "route_pages", "route_pages_group",
     "sparse_attention", "fuse_out_factor", "out_projection",
-    "SequenceCache", "prefill", "decode_step", "num_pages",
+    "SequenceCache", "prefill", "decode_step", "num_pages", "fit_value_factors", "output_error",
 ]
 
 
@@ -332,3 +332,97 @@ def decode_step(cache: SequenceCache, k_new, v_new, q, A, P, E, G, top_k: int, r
         o_lat[h] = o
     y = out_projection(o_lat, G)
     return {"sel": sels, "scores": scores, "o_lat": o_lat, "weight_sums": np.array(wsum), "y": y}
+
+
+# --------------------------------------------------------------------------
+# calibration: Value factors fitted against the complete attention output
+# --------------------------------------------------------------------------
+# The explainer's section "联合优化而非逐分区拟合" (and the BasisKV abstract)
+# contrast two ways of fitting the low-rank factors when the heads are split
+# over tensor-parallel partitions: each partition fitting its own (partial)
+# attention output in isolation, or all partitions' factors optimised together
+# against the complete attention output.  With the Value factor bound to the
+# output projection, head h (KV group g) contributes Z_h A_g B_g W_O,h to the
+# layer output, where Z_h holds the head's exact attention outputs (softmax-
+# weighted raw values) on calibration queries; the target is sum_h Z_h W_O,h.
+
+def output_error(Z, W_O, A, B, heads=None):
+    """Squared Frobenius error of sum_h Z_h A_g B_g W_O,h against sum_h Z_h W_O,h.
+
+    Z: [Hq, N, d]; W_O: [Hq*d, hidden]; A: [Hkv, d, r]; B: [Hkv, r, d];
+    heads: the heads summed (default: all).  g(h) = h // (Hq / Hkv).
+    """
+    Hq, N, d = Z.shape
+    group = Hq // A.shape[0]
+    heads = range(Hq) if heads is None else heads
+    err = np.zeros((N, W_O.shape[1]))
+    for h in heads:
+        g = h // group
+        W = W_O[h * d:(h + 1) * d]
+        err += Z[h] @ W - Z[h] @ A[g] @ B[g] @ W
+    return float(np.sum(err * err))
+
+
+def _lstsq_B(us, Ws, t):
+    """argmin_B || t - sum_i us[i] B Ws[i] ||_F  (design matrix written out, np.linalg.lstsq)."""
+    D = sum(np.kron(u, W.T) for u, W in zip(us, Ws))
+    x = np.linalg.lstsq(D, t.reshape(-1), rcond=None)[0]
+    return x.reshape(us[0].shape[1], Ws[0].shape[0])
+
+
+def _lstsq_A(Zs, Ms, t):
+    """argmin_A || t - sum_i Zs[i] A Ms[i] ||_F  (design matrix written out, np.linalg.lstsq)."""
+    D = sum(np.kron(z, M.T) for z, M in zip(Zs, Ms))
+    x = np.linalg.lstsq(D, t.reshape(-1), rcond=None)[0]
+    return x.reshape(Zs[0].shape[1], Ms[0].shape[0])
+
+
+def fit_value_factors(Z, W_O, num_kv_heads: int, partitions, rank: int, sweeps: int, objective: str):
+    """Low-rank Value factors A_g [d, r], B_g [r, d] of every KV group.
+
+    Z: [Hq, N, d] attention outputs of every query head on N calibration
+    queries; W_O: [Hq*d, hidden]; partitions: lists of KV groups (the
+    tensor-parallel ranks).  Start: A_g = the top-`rank` right singular
+    vectors of the group's stacked Z rows, B_g = A_g^T (a per-partition SVD).
+    Each sweep visits the groups in order; for group g the target is
+
+      "joint":    the complete output, sum over all heads of Z_h W_O,h, minus
+                  the current approximations of every other group's heads;
+      "isolated": the same restricted to the heads of g's own partition,
+
+    and the update solves the linear least-squares problem for B_g with A_g
+    fixed, then for A_g with the new B_g fixed.  Returns (A, B, the complete-
+    output error after the start and after every sweep).
+    """
+    Hq, N, d = Z.shape
+    group = Hq // num_kv_heads
+    hidden = W_O.shape[1]
+    W = [W_O[h * d:(h + 1) * d] for h in range(Hq)]
+    A = np.zeros((num_kv_heads, d, rank))
+    B = np.zeros((num_kv_heads, rank, d))
+    for g in range(num_kv_heads):
+        rows = np.concatenate([Z[h] for h in range(g * group, (g + 1) * group)])
+        Vt = np.linalg.svd(rows, full_matrices=False)[2]
+        A[g] = Vt[:rank].T
+        B[g] = Vt[:rank]
+    part_of = {g: tuple(p) for p in partitions for g in p}
+    history = [output_error(Z, W_O, A, B)]
+    for _ in range(sweeps):
+        for g in range(num_kv_heads):
+            if objective == "joint":
+                scope = range(Hq)
+            elif objective == "isolated":
+                scope = [h for h in range(Hq) if h // group in part_of[g]]
+            else:
+                raise ValueError(f"objective must be 'joint' or 'isolated', not {objective!r}")
+            t = np.zeros((N, hidden))
+            for h in scope:
+                t += Z[h] @ W[h]
+                if h // group != g:
+                    t -= Z[h] @ A[h // group] @ B[h // group] @ W[h]
+            own = range(g * group, (g + 1) * group)
+            B[g] = _lstsq_B([Z[h] @ A[g] for h in own], [W[h] for h in own], t)
+            A[g] = _lstsq_A([Z[h] for h in own], [B[g] @ W[h] for h in own], t)
+        history.append(output_error(Z, W_O, A, B))
+    return A, B, np.array(history)
+

@@ -14,6 +14,7 @@ from tests.test_oracle_pins import ALL_CHECKS
 
 _orig = {name: getattr(ORACLE, name) for name in
          ["append_latents", "page_summaries", "route_pages", "route_pages_group", "sparse_attention",
+          "fit_value_factors", "_lstsq_B", "_lstsq_A",
           "fuse_out_factor", "out_projection", "round_storage", "_round_bf16"]}
 
 
@@ -118,6 +119,47 @@ def _group_sum_as_mean(qs, S, top_k, reduce):
     return sel, (sc / len(qs) if reduce == "sum" else sc)
 
 
+def _lstsq_B_untransposed(us, Ws, t):
+    D = sum(np.kron(u, W) for u, W in zip(us, Ws))
+    x = np.linalg.lstsq(D, t.reshape(-1), rcond=None)[0]
+    return x.reshape(us[0].shape[1], Ws[0].shape[0])
+
+
+def _lstsq_A_drops_last_term(Zs, Ms, t):
+    return _orig["_lstsq_A"](Zs[:1], Ms[:1], t) if len(Zs) > 1 else _orig["_lstsq_A"](Zs, Ms, 0.5 * t)
+
+
+def _fit_with(init_last: bool = False, keep_others: bool = False):
+    """fit_value_factors with one planted change (see MUTATIONS)."""
+    def fit(Z, W_O, num_kv_heads, partitions, rank, sweeps, objective):
+        Hq, N, d = Z.shape
+        group = Hq // num_kv_heads
+        W = [W_O[h * d:(h + 1) * d] for h in range(Hq)]
+        A = np.zeros((num_kv_heads, d, rank))
+        B = np.zeros((num_kv_heads, rank, d))
+        for g in range(num_kv_heads):
+            rows = np.concatenate([Z[h] for h in range(g * group, (g + 1) * group)])
+            Vt = np.linalg.svd(rows, full_matrices=False)[2]
+            sel = Vt[-rank:] if init_last else Vt[:rank]
+            A[g], B[g] = sel.T, sel
+        part_of = {g: tuple(p) for p in partitions for g in p}
+        hist = [ORACLE.output_error(Z, W_O, A, B)]
+        for _ in range(sweeps):
+            for g in range(num_kv_heads):
+                scope = range(Hq) if objective == "joint" else [h for h in range(Hq) if h // group in part_of[g]]
+                t = np.zeros((N, W_O.shape[1]))
+                for h in scope:
+                    t += Z[h] @ W[h]
+                    if h // group != g and not keep_others:
+                        t -= Z[h] @ A[h // group] @ B[h // group] @ W[h]
+                own = range(g * group, (g + 1) * group)
+                B[g] = ORACLE._lstsq_B([Z[h] @ A[g] for h in own], [W[h] for h in own], t)
+                A[g] = ORACLE._lstsq_A([Z[h] for h in own], [B[g] @ W[h] for h in own], t)
+            hist.append(ORACLE.output_error(Z, W_O, A, B))
+        return A, B, np.array(hist)
+    return fit
+
+
 def _outproj_first_head_only(o_lat, G):
     return o_lat[0] @ G[0]
 
@@ -142,6 +184,10 @@ MUTATIONS = {
     "group_route_first_head_only": ("route_pages_group", _group_first_head_only),
     "group_route_max_as_min": ("route_pages_group", _group_max_as_min),
     "group_route_sum_as_mean": ("route_pages_group", _group_sum_as_mean),
+    "fit_start_from_smallest_directions": ("fit_value_factors", _fit_with(init_last=True)),
+    "fit_target_keeps_other_groups_outputs": ("fit_value_factors", _fit_with(keep_others=True)),
+    "fit_B_step_untransposed_W_O": ("_lstsq_B", _lstsq_B_untransposed),
+    "fit_A_step_drops_a_head": ("_lstsq_A", _lstsq_A_drops_last_term),
     "attention_missing_sqrt_d": ("sparse_attention", _attn_no_scale),
     "attention_skips_partial_page": ("sparse_attention", _attn_skip_partial_page),
     "fuse_wrong_head_group": ("fuse_out_factor", _fuse_wrong_group),

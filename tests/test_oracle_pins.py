@@ -512,6 +512,85 @@ def test_incremental_equals_batch():
     check_incremental_equals_batch(ORACLE)
 
 
+# ---------------------------------------------------------------------------
+# calibration: Value factors against the complete attention output
+# ---------------------------------------------------------------------------
+def check_fit_eckart_young(o):
+    """One head, W_O = I: the best rank-r factors give the Eckart-Young error
+    (sum of the squared singular values past r), from the start and after sweeps."""
+    rng = np.random.default_rng(21)
+    N, d, r = 60, 7, 3
+    Z = rng.standard_normal((1, N, d)) * np.array([5.0, 3, 2, 1.5, 1, 0.5, 0.2])
+    sv = np.linalg.svd(Z[0], compute_uv=False)
+    ey = float(np.sum(sv[r:] ** 2))
+    for objective in ("joint", "isolated"):
+        A, B, hist = o.fit_value_factors(Z, np.eye(d), 1, [[0]], r, 0, objective)
+        assert abs(hist[0] - ey) <= 1e-9 * ey
+        A, B, hist = o.fit_value_factors(Z, np.eye(d), 1, [[0]], r, 4, objective)
+        assert np.all(np.abs(hist - ey) <= 1e-8 * ey)
+        assert abs(o.output_error(Z, np.eye(d), A, B) - ey) <= 1e-8 * ey
+
+
+def check_fit_exact_low_rank(o):
+    """Each group's attention outputs lie in an r-dimensional subspace: the
+    factors reproduce the complete output exactly under both objectives."""
+    rng = np.random.default_rng(22)
+    Hq, Hkv, N, d, r, hid = 4, 2, 50, 6, 2, 9
+    basis = [np.linalg.qr(rng.standard_normal((d, r)))[0] for _ in range(Hkv)]
+    Z = np.stack([rng.standard_normal((N, r)) @ basis[h // 2].T for h in range(Hq)])
+    W_O = rng.standard_normal((Hq * d, hid))
+    scale = o.output_error(Z, W_O, np.zeros((Hkv, d, r)), np.zeros((Hkv, r, d)))
+    for objective in ("joint", "isolated"):
+        A, B, hist = o.fit_value_factors(Z, W_O, Hkv, [[0], [1]], r, 2, objective)
+        assert hist[-1] <= 1e-20 * scale
+
+
+def check_fit_least_squares_steps(o):
+    """One term: the B and A updates equal the two-sided least-squares closed forms."""
+    rng = np.random.default_rng(23)
+    N, r, d, hid = 30, 3, 5, 8
+    U = rng.standard_normal((N, r))
+    W = rng.standard_normal((d, hid))
+    t = rng.standard_normal((N, hid))
+    want_B = np.linalg.solve(U.T @ U, U.T @ t @ W.T) @ np.linalg.inv(W @ W.T)
+    np.testing.assert_allclose(o._lstsq_B([U], [W], t), want_B, atol=1e-10)
+    Zs = rng.standard_normal((N, d))
+    M = rng.standard_normal((r, hid))
+    want_A = np.linalg.solve(Zs.T @ Zs, Zs.T @ t @ M.T) @ np.linalg.inv(M @ M.T)
+    np.testing.assert_allclose(o._lstsq_A([Zs], [M], t), want_A, atol=1e-10)
+
+
+def check_fit_sweeps(o):
+    """Joint sweeps never increase the complete-output error (each update is an
+    exact minimisation of it); with one partition the two objectives coincide."""
+    rng = np.random.default_rng(24)
+    Hq, Hkv, N, d, r, hid = 6, 3, 40, 5, 2, 8
+    Z = rng.standard_normal((Hq, N, d))
+    W_O = rng.standard_normal((Hq * d, hid))
+    _, _, hist = o.fit_value_factors(Z, W_O, Hkv, [[0], [1], [2]], r, 6, "joint")
+    assert np.all(np.diff(hist) <= 1e-9 * hist[0])
+    assert hist[-1] < 0.9 * hist[0]
+    _, _, h1 = o.fit_value_factors(Z, W_O, Hkv, [[0, 1, 2]], r, 3, "isolated")
+    _, _, h2 = o.fit_value_factors(Z, W_O, Hkv, [[0, 1, 2]], r, 3, "joint")
+    np.testing.assert_allclose(h1, h2, rtol=1e-12)
+
+
+def test_fit_eckart_young():
+    check_fit_eckart_young(ORACLE)
+
+
+def test_fit_exact_low_rank():
+    check_fit_exact_low_rank(ORACLE)
+
+
+def test_fit_least_squares_steps():
+    check_fit_least_squares_steps(ORACLE)
+
+
+def test_fit_sweeps():
+    check_fit_sweeps(ORACLE)
+
+
 ALL_CHECKS = [
     check_bf16_rounding, check_append_identity, check_append_projection,
     check_summary_closed_form, check_summary_low_rank_residual,
@@ -521,4 +600,5 @@ ALL_CHECKS = [
     check_out_projection_associativity, check_decode_dense_special_case,
     check_decode_all_pages_real_factors, check_new_token_is_attended, check_golden,
     check_incremental_equals_batch,
+    check_fit_eckart_young, check_fit_exact_low_rank, check_fit_least_squares_steps, check_fit_sweeps,
 ]
