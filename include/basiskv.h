@@ -174,7 +174,7 @@ BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basis
  * bf16 ulp from basiskv_append's correctly rounded fp64 result where the two
  * straddle a rounding midpoint.  The summaries of every touched page are then
  * recomputed in fp64 from the stored C and R, as basiskv_append does.
- * Requires head_dim 64 or 128, rank_v a multiple of 16 in [16, 128], rank_k a
+ * Requires head_dim 128, rank_v a multiple of 16 in [16, 128], rank_k a
  * multiple of 16 in [16, 64] (else BASISKV_ERR_UNSUPPORTED); k_new and v_new
  * 16-byte aligned.  Work is split in tiles of 128 consecutive new tokens per
  * (sequence, KV head), so short appends leave most of the GPU idle.

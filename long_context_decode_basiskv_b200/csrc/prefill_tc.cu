@@ -399,7 +399,9 @@ __global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams 
 }
 
 bool prefill_tc_supported(bool bf16, int d, int r, int s) {
-  return bf16 && (d == 64 || d == 128) && r >= 16 && r <= 128 && r % 16 == 0 && s >= 16 && s <= 64 &&
+  // head_dim 128 only: the shapes the parity tests exercise (64 would take the same code with one
+  // K atom per operand, and is left to basiskv_append until it is tested)
+  return bf16 && d == 128 && r >= 16 && r <= 128 && r % 16 == 0 && s >= 16 && s <= 64 &&
          s % 16 == 0 && pf_layout(d, r, s).total + 1024 <= 227 * 1024;
 }
 

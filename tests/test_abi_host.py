@@ -178,7 +178,8 @@ def test_prefill_checks(L):
     """basiskv_prefill: bf16 with ranks that are multiples of 16 only; otherwise basiskv_append's checks."""
     good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
     f = bk.CFactors(256, 256, 256, 256)
-    for bad in (dict(dtype=bk.F32), dict(rank_k=8), dict(rank_v=24), dict(head_dim=96, rank_v=32)):
+    for bad in (dict(dtype=bk.F32), dict(rank_k=8), dict(rank_v=24), dict(head_dim=96, rank_v=32),
+                dict(head_dim=64, rank_v=32)):
         cfg = _cfg(**bad)
         assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 1, 64, 256,
                                  None) == bk.ERR_UNSUPPORTED, bad
