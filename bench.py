@@ -15,7 +15,12 @@ the roofline of the attention kernel.  L2 is flushed before every step by
 reading a 256 MiB buffer (outside the events).
 
 With N > 1 (torchrun, one process per GPU) every rank runs an independent
-replica on its own sequences (weak scaling; the path has no exchange step).
+replica on its own sequences (weak scaling; the path has no exchange step);
+``--tp`` instead shards the heads of one workload over the ranks and adds one
+NCCL all-reduce of the layer output per step (strong scaling).
+``--routing group_sum|group_max`` routes once per KV group instead of once per
+query head.  After the decode measurements the line also reports the prefill
+append of the whole context (tensor-core path and fp64 path; ``prefill``).
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead.
 """
 from __future__ import annotations
