@@ -90,3 +90,14 @@ def test_gloo_all_reduce_of_partials(tmp_path):
     for r in range(world):
         y = torch.load(tmp_path / f"{r}.pt").numpy()
         np.testing.assert_allclose(y, full, rtol=0, atol=1e-10 * np.abs(full).max())
+
+
+def test_engine_rejects_unknown_modes():
+    """Engine options are checked before any device work."""
+    from long_context_decode_basiskv_b200.engine import DecodeEngine
+
+    case = make_case(WORKLOADS["tiny_fp32"], "cpu")
+    with pytest.raises(ValueError):
+        DecodeEngine(case, device="cpu", routing="per_page")
+    with pytest.raises(ValueError):
+        DecodeEngine(case, device="cpu", prefill_mode="fast")
