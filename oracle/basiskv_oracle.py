@@ -39,8 +39,11 @@ round-to-nearest-even, or fp32) happens exactly where a value is stored.
 Pins (tests/test_oracle_pins.py): dense-attention special case against
 torch's scaled_dot_product_attention, identity factors, closed-form page
 means, a full-sort and brute-force check of the selection, softmax weights
-summing to one, associativity of the fused out-projection, and a hand-worked
-golden example.  Every function below is pinned by at least one of them.
+summing to one, associativity of the fused out-projection, a hand-worked
+golden example; for the per-group routing a hand-worked two-head example and
+reductions to per-head routing; for the factor fit the Eckart-Young error,
+exact low-rank recovery, closed-form least-squares steps and monotone sweeps.
+Every function below is pinned by at least one of them.
 """
 from __future__ import annotations
 
