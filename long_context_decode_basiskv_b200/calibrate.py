@@ -24,7 +24,11 @@ N x hidden x r x d is formed.  Runs on whatever device the tensors are on
 """
 from __future__ import annotations
 
+import dataclasses
+
 import torch
+
+from .workloads import Case, gram_matrices, key_factors_from_grams
 
 
 def output_error(Z: torch.Tensor, W_O: torch.Tensor, A: torch.Tensor, B: torch.Tensor) -> float:
@@ -108,3 +112,17 @@ def calibration_outputs(q: torch.Tensor, keys: torch.Tensor, values: torch.Tenso
         s = (q[:, h] @ keys[:, g].T) / d ** 0.5
         out[h] = torch.softmax(s, dim=-1) @ values[:, g]
     return out
+
+
+def with_value_factors(case: Case, A: torch.Tensor, B: torch.Tensor) -> Case:
+    """`case` with the Value factors A [Hkv, d, r] and B [Hkv, r, d] (for instance from
+    fit_value_factors) and the key factors refitted to them as the workloads fit them:
+    P_g by least squares of K on C = V A_g, E_g the top rank_k directions of the
+    residual, over every token of the case.  All four are rounded to the case's
+    storage dtype, so the decode path (basiskv_fuse_out_factor builds G_h = B_g W_O,h)
+    runs on them directly."""
+    gvv, gvk, gkk = gram_matrices(case.keys, case.values)
+    P, E = key_factors_from_grams(gvv, gvk, gkk, A.detach().to("cpu", torch.float64), case.wl.rank_k)
+    td, dev = case.A.dtype, case.A.device
+    return dataclasses.replace(case, A=A.to(dev, td), Bf=B.to(dev, td), P=P.to(dev, td), E=E.to(dev, td))
+

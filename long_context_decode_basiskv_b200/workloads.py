@@ -249,6 +249,19 @@ def _fit_factors(wl: Workload, keys, values):
     fp64 copy of the cache.
     """
     Hkv, d, r, s = wl.num_kv_heads, wl.head_dim, wl.rank_v, wl.rank_k
+    gvv, gvk, gkk = gram_matrices(keys, values)
+    A = torch.zeros((Hkv, d, r), dtype=torch.float64)
+    for h in range(Hkv):
+        A[h] = _top_eigvecs(gvv[h], r)                   # d x r
+    Pm, E = key_factors_from_grams(gvv, gvk, gkk, A, s)
+    Bf = A.transpose(1, 2).contiguous()
+    return A, Bf, Pm, E
+
+
+def gram_matrices(keys, values):
+    """Per-KV-head fp64 Gram matrices V^T V, V^T K, K^T K over every token of the
+    given sequences (lists of [T, Hkv, d]), accumulated in chunks; on the host."""
+    Hkv, d = keys[0].shape[1], keys[0].shape[2]
     dev = keys[0].device
     gvv = torch.zeros((Hkv, d, d), dtype=torch.float64, device=dev)
     gvk = torch.zeros_like(gvv)
@@ -260,20 +273,24 @@ def _fit_factors(wl: Workload, keys, values):
             gvv += torch.einsum("thd,the->hde", v, v)
             gvk += torch.einsum("thd,the->hde", v, k)
             gkk += torch.einsum("thd,the->hde", k, k)
-    gvv, gvk, gkk = gvv.cpu(), gvk.cpu(), gkk.cpu()
-    A = torch.zeros((Hkv, d, r), dtype=torch.float64)
+    return gvv.cpu(), gvk.cpu(), gkk.cpu()
+
+
+def key_factors_from_grams(gvv, gvk, gkk, A, s: int):
+    """Key factors for given Value encoders A [Hkv, d, r]: P_g by least squares of K on
+    C = V A_g, E_g the top-s directions of the residual K - C P_g (from the Gram matrices)."""
+    Hkv, d, r = A.shape
     Pm = torch.zeros((Hkv, r, d), dtype=torch.float64)
     E = torch.zeros((Hkv, d, s), dtype=torch.float64)
     for h in range(Hkv):
-        a = _top_eigvecs(gvv[h], r)                      # d x r
+        a = A[h].to(torch.float64)
         ctc = a.T @ gvv[h] @ a                           # C^T C
         ctk = a.T @ gvk[h]                               # C^T K
         p = torch.linalg.solve(ctc, ctk)                 # r x d
         res = gkk[h] - ctk.T @ p - p.T @ ctk + p.T @ ctc @ p
         res = 0.5 * (res + res.T)
-        A[h], Pm[h], E[h] = a, p, _top_eigvecs(res, s)
-    Bf = A.transpose(1, 2).contiguous()
-    return A, Bf, Pm, E
+        Pm[h], E[h] = p, _top_eigvecs(res, s)
+    return Pm, E
 
 
 def _plant_hot_pages(wl: Workload, rng, q32, keys32, lengths):

@@ -54,3 +54,40 @@ def test_calibration_outputs_match_oracle_attention():
         for n in range(N):
             o, _, _ = O.sparse_attention(q[n, h], K[:, g], V[:, g], np.arange(O.num_pages(T, 4)), 4)
             np.testing.assert_allclose(Z[h, n], o, atol=1e-12)
+
+
+def test_with_value_factors_refits_the_key_factors_like_the_workloads():
+    """Given the workloads' own (unrounded) Value encoders, the refit reproduces their P and E."""
+    from long_context_decode_basiskv_b200.workloads import WORKLOADS, _top_eigvecs, gram_matrices, make_case, shrink
+
+    for wl in (WORKLOADS["tiny_fp32"], shrink(WORKLOADS["llama3_8b_32k"], batch=2, context=700, name="cal")):
+        case = make_case(wl, "cpu")
+        gvv, _, _ = gram_matrices(case.keys, case.values)
+        A = torch.stack([_top_eigvecs(gvv[h], wl.rank_v) for h in range(wl.num_kv_heads)])
+        out = CAL.with_value_factors(case, A, A.transpose(1, 2))
+        for a, b in ((out.A, case.A), (out.Bf, case.Bf), (out.P, case.P), (out.E, case.E)):
+            assert a.dtype == b.dtype and torch.equal(a, b)
+
+
+def test_calibrated_case_runs_through_the_oracle():
+    """Joint factors fitted on calibration outputs of a case, then one oracle decode step on it."""
+    from long_context_decode_basiskv_b200.workloads import WORKLOADS, make_case
+
+    case = make_case(WORKLOADS["tiny_fp32"], "cpu")
+    wl = case.wl
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn((64, wl.num_q_heads, wl.head_dim), generator=g, dtype=torch.float64) * 2
+    K = case.keys[0].to(torch.float64)
+    V = case.values[0].to(torch.float64)
+    Z = CAL.calibration_outputs(q, K, V)
+    W = case.W_O.to(torch.float64)
+    A, B, hist = CAL.fit_value_factors(Z, W, wl.num_kv_heads, [[0], [1]], wl.rank_v, 2, "joint")
+    assert hist[-1] <= hist[0]
+    cal = CAL.with_value_factors(case, A, B)
+    f64 = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    G = O.fuse_out_factor(f64(cal.Bf), f64(cal.W_O), wl.num_q_heads, "f32")
+    cache = O.prefill(f64(K)[:-1], f64(V)[:-1], f64(cal.A), f64(cal.P), f64(cal.E), wl.page_size, "f32",
+                      capacity=K.shape[0])
+    out = O.decode_step(cache, f64(K)[-1], f64(V)[-1], f64(case.q[0]), f64(cal.A), f64(cal.P), f64(cal.E), G,
+                        wl.top_k)
+    assert np.all(np.isfinite(out["y"])) and np.allclose(out["weight_sums"], 1.0)
