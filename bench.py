@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from long_context_decode_basiskv_b200.workloads import WORKLOADS, make_case  # noqa: E402
+from long_context_decode_basiskv_b200.workloads import WORKLOADS, make_case, shrink  # noqa: E402
 
 METRIC = "decode tokens/s per layer on 1 B200; route+attn HBM GB/s vs ~8 TB/s roofline"
 UNIT = "tokens/s"
@@ -60,11 +60,15 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="llama3_8b_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--context", type=int, default=None,
+                    help="tokens per sequence instead of the workload's (a smaller case of the same "
+                         "kernels, for profiling; a ragged workload becomes uniform)")
     ap.add_argument("--routing", default="head", choices=["head", "group_sum", "group_max"],
                     help="one page selection per query head (the method as stated), or per KV group")
-    ap.add_argument("--oracle-seqs", type=int, default=2, help="sequences in the CPU-baseline sample")
-    ap.add_argument("--oracle-repeats", type=int, default=100,
-                    help="decode steps per sampled sequence in the CPU baseline (about 10 s in total)")
+    ap.add_argument("--oracle-repeats", type=int, default=200,
+                    help="decode steps per host process in the CPU baseline, at most")
+    ap.add_argument("--oracle-budget", type=float, default=3.0,
+                    help="seconds each host process spends on decode steps in the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-append measurement")
@@ -93,6 +97,14 @@ def init_dist(world, backend):
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
+
+
+def chosen_workload(args):
+    """The named workload, or a shorter-context case of it (--context)."""
+    wl = WORKLOADS[args.workload]
+    if args.context is not None:
+        wl = dataclasses.replace(shrink(wl, context=args.context, name=f"{wl.name}@{args.context}"), ragged=None)
+    return wl
 
 
 def replica_workload(wl, rank: int, world: int):
@@ -166,7 +178,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
         names = [k for k, v in self.REASONS.items() if self.reasons & v and k != "gpu_idle"]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                "window": "warm-up, timed steps, per-phase pass and end-to-end pass"}
 
 
 # ---------------------------------------------------------------------------
@@ -225,43 +238,158 @@ def profiled_traffic(kernel_file: str):
 
 
 # ---------------------------------------------------------------------------
-# CPU baseline: the oracle on a bounded sample
+# CPU baseline: the oracle on a bounded sample, on every host core
 # ---------------------------------------------------------------------------
-def oracle_sample(case, nseq: int, repeats: int = 1, routing: str = "head"):
-    """Time the oracle's decode step (append .. out-projection) on `nseq` sequences.
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover - not Linux
+        return os.cpu_count() or 1
 
-    The prefill of each sequence's oracle cache is untimed.  A repeat re-runs
-    the same decode step (the cache length is reset before the append).
-    Returns (seconds per decode step list, description).
-    """
+
+def _oracle_worker(conn, path: str, b: int, wl_fields: dict, routing: str):
+    """One host process: load sequence b of the dumped case, build its oracle
+    cache (untimed), then on each request run `repeats` decode steps of that
+    sequence and send back (start, end, per-step seconds)."""
     from threadpoolctl import threadpool_limits
 
     from oracle import basiskv_oracle as O
 
-    wl = case.wl
-    storage = "f32" if wl.dtype == "f32" else "bf16"
-
-    def f64(t):
-        return t.detach().to("cpu").to(torch.float64).numpy()
-
-    A, P, E = f64(case.A), f64(case.P), f64(case.E)
-    times = []
     with threadpool_limits(1):
-        G = O.fuse_out_factor(f64(case.Bf), f64(case.W_O), wl.num_q_heads, storage)
-        for b in range(min(nseq, wl.batch)):
-            K, V = f64(case.keys[b]), f64(case.values[b])
-            L = K.shape[0]
-            cache = O.prefill(K[:-1], V[:-1], A, P, E, wl.page_size, storage, capacity=L)
-            q = f64(case.q[b])
-            for _ in range(repeats):
+        storage = wl_fields["storage"]
+        fac = np.load(os.path.join(path, "factors.npz"))
+        A, P, E = (fac[k].astype(np.float64) for k in ("A", "P", "E"))
+        G = O.fuse_out_factor(fac["Bf"].astype(np.float64), fac["W_O"].astype(np.float64),
+                              wl_fields["num_q_heads"], storage)
+        seq = np.load(os.path.join(path, f"seq{b}.npz"))
+        K, V, q = (seq[k].astype(np.float64) for k in ("K", "V", "q"))
+        L = K.shape[0]
+        cache = O.prefill(K[:-1], V[:-1], A, P, E, wl_fields["page_size"], storage, capacity=L)
+        conn.send("ready")
+        while True:
+            req = conn.recv()
+            if req is None:
+                break
+            repeats, budget = req
+            times = []
+            t_start = time.perf_counter()
+            while len(times) < repeats and (budget is None or time.perf_counter() - t_start < budget):
                 cache.length = L - 1
                 t0 = time.perf_counter()
-                O.decode_step(cache, K[-1], V[-1], q, A, P, E, G, wl.top_k, routing=routing)
+                O.decode_step(cache, K[-1], V[-1], q, A, P, E, G, wl_fields["top_k"], routing=routing)
                 times.append(time.perf_counter() - t0)
-    desc = (f"fp64 numpy oracle, 1 thread: decode step (append, summary, {routing} route, attention, "
-            f"out-projection) of {min(nseq, wl.batch)} of the {wl.batch} sequences x {repeats}, "
-            f"prefill untimed")
-    return times, desc
+            conn.send((t_start, time.perf_counter(), times))
+    conn.close()
+
+
+class OracleHost:
+    """The fp64 oracle on the host cores: one spawned process per core, each
+    decoding one sequence of the case (sequence i mod B on process i), with
+    one BLAS thread each.  The case's tensors travel through files in a
+    temporary directory (storage values, converted exactly to fp64 by the
+    workers).  Processes are capped by free host memory."""
+
+    def __init__(self, case, routing: str = "head", workers: int | None = None):
+        import multiprocessing as mp
+        import tempfile
+
+        wl = case.wl
+        self.wl, self.routing = wl, routing
+        cores = host_cores()
+        L_max = max(case.lengths)
+        per_worker = (L_max * wl.num_kv_heads * 8 * (3 * wl.head_dim + wl.rank_v + wl.rank_k)
+                      + wl.num_q_heads * wl.rank_v * wl.hidden * 8 * 2 + (256 << 20))
+        try:
+            import psutil
+            mem_cap = max(1, int(psutil.virtual_memory().available * 0.5 // per_worker))
+        except Exception:  # noqa: BLE001
+            mem_cap = cores
+        self.workers = max(1, min(workers or cores, cores, mem_cap))
+        self.dir = tempfile.mkdtemp(prefix="bkv_oracle_", dir="/dev/shm" if os.path.isdir("/dev/shm") else None)
+
+        def f32(t):
+            return t.detach().to("cpu", torch.float32).numpy()
+
+        np.savez(os.path.join(self.dir, "factors.npz"), A=f32(case.A), P=f32(case.P), E=f32(case.E),
+                 Bf=f32(case.Bf), W_O=f32(case.W_O))
+        seqs = sorted({i % wl.batch for i in range(self.workers)})
+        for b in seqs:
+            np.savez(os.path.join(self.dir, f"seq{b}.npz"), K=f32(case.keys[b]), V=f32(case.values[b]),
+                     q=f32(case.q[b]))
+        fields = {"storage": "f32" if wl.dtype == "f32" else "bf16", "num_q_heads": wl.num_q_heads,
+                  "page_size": wl.page_size, "top_k": wl.top_k}
+        ctx = mp.get_context("spawn")
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        self.procs, self.conns = [], []
+        try:
+            for i in range(self.workers):
+                parent, child = ctx.Pipe()
+                p = ctx.Process(target=_oracle_worker, args=(child, self.dir, i % wl.batch, fields, routing),
+                                daemon=True)
+                p.start()
+                self.procs.append(p)
+                self.conns.append(parent)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        for c in self.conns:
+            if c.recv() != "ready":
+                raise RuntimeError("oracle worker failed to start")
+
+    def run(self, repeats: int, workers: int | None = None, budget: float | None = None):
+        """Up to `repeats` decode steps (stopping after `budget` seconds, if given) on
+        each of the first `workers` processes at once.  Returns (steps, wall seconds
+        from the first start to the last end, all step times)."""
+        use = self.conns[:workers or self.workers]
+        for c in use:
+            c.send((repeats, budget))
+        res = [c.recv() for c in use]
+        wall = max(r[1] for r in res) - min(r[0] for r in res)
+        times = [t for r in res for t in r[2]]
+        return len(times), wall, times
+
+    def close(self):
+        import shutil
+
+        for c in self.conns:
+            try:
+                c.send(None)
+            except Exception:  # noqa: BLE001
+                pass
+        for p in self.procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.terminate()
+        shutil.rmtree(self.dir, ignore_errors=True)
+
+    def describe(self, what: str) -> str:
+        wl = self.wl
+        return (f"fp64 numpy oracle on {self.workers} host processes (1 BLAS thread each; "
+                f"{host_cores()} cores available): process i decodes sequence i mod {wl.batch} of the "
+                f"workload, {what} (decode step = append, summary, {self.routing} route, attention, "
+                f"out-projection), prefill untimed; value = decode steps / wall time")
+
+
+def cpu_baseline(case, routing: str, repeats: int, budget: float):
+    """The oracle on all host cores (throughput of independent decode steps), plus
+    the same decode step on one core alone.  Each process runs up to `repeats`
+    steps and stops after `budget` seconds."""
+    host = OracleHost(case, routing)
+    try:
+        n1, w1, _ = host.run(repeats, workers=1, budget=budget)
+        steps, wall, _ = host.run(repeats, budget=budget)
+    finally:
+        host.close()
+    return {"value": round(steps / wall, 3), "unit": UNIT, "cores": host.workers, "kind": "oracle",
+            "sample": host.describe(f"{steps // host.workers} decode steps per process"),
+            "seconds": round(wall, 3), "cpu_seconds": round(wall * host.workers, 1),
+            "single_thread": {"value": round(n1 / w1, 3), "unit": UNIT, "cores": 1,
+                              "sample": f"one process alone: {n1} decode steps of sequence 0"}}
 
 
 # ---------------------------------------------------------------------------
@@ -325,12 +453,12 @@ def run_ours(args, world, rank, local):
     if args.tp:
         from long_context_decode_basiskv_b200.tensor_parallel import reduce_y, shard_case
 
-        full_wl = WORKLOADS[args.workload]
+        full_wl = chosen_workload(args)
         case = shard_case(make_case(full_wl, dev), rank, world)   # every rank builds the same case
         wl = case.wl
         tokens_per_step = full_wl.batch                           # the ranks share one batch
     else:
-        full_wl = wl = replica_workload(WORKLOADS[args.workload], rank, world)
+        full_wl = wl = replica_workload(chosen_workload(args), rank, world)
         case = make_case(wl, dev)
         tokens_per_step = world * wl.batch                        # independent replicas
 
@@ -377,73 +505,76 @@ def run_ours(args, world, rank, local):
                     evs.append(e)
         return evs
 
-    run_steps(args.warmup, False, ["step"])
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    # clocks are sampled over the whole measurement (warm-up, timed steps, per-phase
+    # pass, end-to-end pass): the timed region alone is too short for NVML's rate
+    clk = ClockSampler(local, period_s=0.0005)
+    with clk:
+        run_steps(args.warmup, False, ["step"])
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
         evs = run_steps(args.steps, True, ["step"])
         torch.cuda.synchronize()
-    barrier(world)
-    step_ms = [ev[0].elapsed_time(ev[1]) for ev in evs]
-    total_ms = max_over_ranks(sum(step_ms), world, dev)
-    # per-phase breakdown (separate pass; not part of the headline number)
-    run_steps(max(3, args.warmup), False, order)
-    evs = run_steps(min(args.steps, 100), True, order)
-    torch.cuda.synchronize()
-    per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, name in enumerate(order)}
-    ms_per_step = total_ms / args.steps
-    value = tokens_per_step * args.steps / (total_ms / 1e3)
-
-    mean = {k: sum(v) / len(v) for k, v in per.items()}
-    peak, peak_kind = measured_peak()
-    attn_gbs = nbytes["decode_attn"] / (mean["decode_attn"] * 1e-3) / 1e9
-    ra_gbs = (nbytes["route"] + nbytes["decode_attn"]) / ((mean["append_route"] + mean["decode_attn"]) * 1e-3) / 1e9
-    # the committed counters are for per-head routing (other routings read other pages)
-    traffic_rec = profiled_traffic("decode_attn.cu") if args.routing == "head" else None
-    roofline = {
-        "kernel": "basiskv_decode_attn (one launch: union slice, attention, split merge)",
-        "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
-        "frac": round(attn_gbs / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-        "algorithmic_bytes": nbytes["decode_attn"],
-        "traffic": traffic_rec["dram_bytes_per_launch"] if traffic_rec else None,
-    }
-
-    # end to end through the public API: pinned host inputs -> step -> host output
-    e2e = None
-    if not args.no_e2e:
-        hin = eng.input_buffer().cpu().pin_memory()   # q, k_new, v_new of the step, packed
-        hy = torch.empty(eng.y.shape, dtype=eng.y.dtype).pin_memory()
-        bi = hin.numel() * hin.element_size()
-        bo = hy.numel() * hy.element_size()
-
-        def e2e_steps(n, record):
-            out = []
-            with torch.cuda.stream(stream):
-                for _ in range(n):
-                    torch.sum(flush, dim=0, out=sink)
-                    if record:
-                        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                        a.record(stream)
-                    eng.input_buffer().copy_(hin, non_blocking=True)
-                    eng.graph_step()
-                    exchange()
-                    hy.copy_(eng.y, non_blocking=True)
-                    if record:
-                        b_.record(stream)
-                        out.append((a, b_))
-            return out
-
-        e2e_steps(max(3, args.warmup), False)
-        torch.cuda.synchronize()
         barrier(world)
-        pairs = e2e_steps(args.steps, True)
+        step_ms = [ev[0].elapsed_time(ev[1]) for ev in evs]
+        total_ms = max_over_ranks(sum(step_ms), world, dev)
+        # per-phase breakdown (separate pass; not part of the headline number)
+        run_steps(max(3, args.warmup), False, order)
+        evs = run_steps(min(args.steps, 100), True, order)
         torch.cuda.synchronize()
-        barrier(world)
-        e2e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in pairs), world, dev)
-        e2e = {"value": round(tokens_per_step * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
-               "ms_per_step": round(e2e_ms / args.steps, 4)}
+        per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, name in enumerate(order)}
+        ms_per_step = total_ms / args.steps
+        value = tokens_per_step * args.steps / (total_ms / 1e3)
+
+        mean = {k: sum(v) / len(v) for k, v in per.items()}
+        peak, peak_kind = measured_peak()
+        attn_gbs = nbytes["decode_attn"] / (mean["decode_attn"] * 1e-3) / 1e9
+        ra_gbs = (nbytes["route"] + nbytes["decode_attn"]) / ((mean["append_route"] + mean["decode_attn"]) * 1e-3) / 1e9
+        # the committed counters are for per-head routing (other routings read other pages)
+        traffic_rec = profiled_traffic("decode_attn.cu") if args.routing == "head" else None
+        roofline = {
+            "kernel": "basiskv_decode_attn (one launch: union slice, attention, split merge)",
+            "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(attn_gbs / peak, 4), "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+            "algorithmic_bytes": nbytes["decode_attn"],
+            "traffic": traffic_rec["dram_bytes_per_launch"] if traffic_rec else None,
+        }
+
+        # end to end through the public API: pinned host inputs -> step -> host output
+        e2e = None
+        if not args.no_e2e:
+            hin = eng.input_buffer().cpu().pin_memory()   # q, k_new, v_new of the step, packed
+            hy = torch.empty(eng.y.shape, dtype=eng.y.dtype).pin_memory()
+            bi = hin.numel() * hin.element_size()
+            bo = hy.numel() * hy.element_size()
+
+            def e2e_steps(n, record):
+                out = []
+                with torch.cuda.stream(stream):
+                    for _ in range(n):
+                        torch.sum(flush, dim=0, out=sink)
+                        if record:
+                            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                            a.record(stream)
+                        eng.input_buffer().copy_(hin, non_blocking=True)
+                        eng.graph_step()
+                        exchange()
+                        hy.copy_(eng.y, non_blocking=True)
+                        if record:
+                            b_.record(stream)
+                            out.append((a, b_))
+                return out
+
+            e2e_steps(max(3, args.warmup), False)
+            torch.cuda.synchronize()
+            barrier(world)
+            pairs = e2e_steps(args.steps, True)
+            torch.cuda.synchronize()
+            barrier(world)
+            e2e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in pairs), world, dev)
+            e2e = {"value": round(tokens_per_step * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
+                   "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                   "ms_per_step": round(e2e_ms / args.steps, 4)}
 
     prefill = None
     if not args.no_prefill:
@@ -451,9 +582,7 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        times, desc = oracle_sample(case, args.oracle_seqs, args.oracle_repeats, args.routing)
-        cpu = {"value": round(len(times) / sum(times), 3), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": desc, "seconds": round(sum(times), 3)}
+        cpu = cpu_baseline(case, args.routing, args.oracle_repeats, args.oracle_budget)
 
     if rank == 0:
         line = {
@@ -491,21 +620,29 @@ def run_ours(args, world, rank, local):
 # reference arm: the fp64 oracle on the host cores
 # ---------------------------------------------------------------------------
 def run_reference(args, world, rank):
+    """The fp64 oracle on the host cores (rank 0 only).  One step = one decode step
+    on every host process at once (process i decodes sequence i mod B)."""
     if rank != 0:
         return
-    wl = WORKLOADS[args.workload]
+    wl = chosen_workload(args)
     case = make_case(wl, "cpu")
-    times, desc = oracle_sample(case, 1, repeats=args.warmup + args.steps, routing=args.routing)
-    timed = times[args.warmup:]
-    value = len(timed) / sum(timed)
+    host = OracleHost(case, args.routing)
+    try:
+        host.run(args.warmup)
+        steps, wall, times = host.run(args.steps)
+    finally:
+        host.close()
+    value = steps / wall
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(1e3 * sum(timed) / len(timed), 3),
+        "warmup": args.warmup, "ms_per_step": round(1e3 * wall / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
         "config": {"workload": wl.name, "batch": wl.batch, "routing": args.routing,
-                   "sample": "one sequence per step"},
-        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+                   "sample": f"one step = one decode step on each of {host.workers} host processes"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": host.workers, "kind": "oracle",
+                         "sample": host.describe(f"{args.warmup} untimed + {args.steps} timed decode steps "
+                                                 f"per process")},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
