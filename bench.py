@@ -556,10 +556,13 @@ def run_ours(args, world, rank, local):
                         if record:
                             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                             a.record(stream)
-                        eng.input_buffer().copy_(hin, non_blocking=True)
-                        eng.graph_step()
-                        exchange()
-                        hy.copy_(eng.y, non_blocking=True)
+                        if args.tp:
+                            eng.input_buffer().copy_(hin, non_blocking=True)
+                            eng.graph_step()
+                            exchange()
+                            hy.copy_(eng.y, non_blocking=True)
+                        else:
+                            eng.graph_step_host(hin, hy)   # copy in, step, copy out: one graph
                         if record:
                             b_.record(stream)
                             out.append((a, b_))

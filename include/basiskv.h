@@ -61,8 +61,9 @@ extern "C" {
 #endif
 
 /* 1: append, route, decode_attn, out_proj and their helpers;
- * 2: adds basiskv_route_group and basiskv_prefill (nothing earlier changed). */
-#define BASISKV_ABI_VERSION 2
+ * 2: adds basiskv_route_group and basiskv_prefill;
+ * 3: decode_attn accepts sel = sel_cnt = NULL (the routing call's selection). */
+#define BASISKV_ABI_VERSION 3
 
 typedef enum {
   BASISKV_OK = 0,
@@ -190,8 +191,13 @@ BASISKV_API basiskv_status basiskv_prefill(const basiskv_config* cfg, const basi
  * logical page.  If n_b <= top_k + 2 every page is selected; otherwise pages
  * 0 and n_b - 1 plus the top_k of pages 1..n_b-2 under the order (score
  * descending, page index ascending).
+ * A NaN score ranks below every other score (NaN pages are kept only when
+ * fewer than top_k others exist, lowest page index first).
  * Outputs (device): sel [batch][Hq][top_k + 2] int32 logical page indices in
- * ascending order, padded with -1; sel_cnt [batch][Hq] int32.
+ * ascending order, padded with -1; sel_cnt [batch][Hq] int32.  The call also
+ * leaves in the workspace, per (sequence, KV head), the ascending union of the
+ * pages its G query heads selected (with their physical page ids), which a
+ * following basiskv_decode_attn with sel = sel_cnt = NULL attends over.
  * scores (device, optional, may be NULL): [batch][Hq][max_pages] fp32, the
  * score of every page p < n_b (others untouched).
  * With scores == NULL the call reads no summary of page 0 or of page n_b - 1
@@ -200,9 +206,12 @@ BASISKV_API basiskv_status basiskv_prefill(const basiskv_config* cfg, const basi
  * two may run concurrently on different streams.
  * workspace (device): at least basiskv_workspace_bytes(cfg, batch, max_pages)
  * bytes, zero-filled once when it is allocated.  It holds per-call scratch
- * plus small counters that every decode_attn call leaves at zero again, so no
- * further clearing is needed between calls (a counter found out of range sets
- * BASISKV_DEVERR_WORKSPACE).  Calls sharing one workspace must not overlap.
+ * plus small counters that every route call leaves at zero again, so no
+ * further clearing is needed between calls of one shape (a counter found out
+ * of range sets BASISKV_DEVERR_WORKSPACE).  The counters' place depends on the
+ * shape: before a workspace serves another (cfg, batch, max_pages), zero-fill
+ * it again.  Calls sharing one workspace must not overlap.  Requires
+ * num_phys_pages < 2^24.
  */
 BASISKV_API basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache,
                              const void* q, int32_t batch, int32_t* sel, int32_t* sel_cnt,
@@ -236,9 +245,17 @@ BASISKV_API basiskv_status basiskv_route_group(const basiskv_config* cfg, const 
  * of the pages in sel[b][h][0 .. sel_cnt-1], s_j = q_h . K_j / sqrt(d) on the
  * original keys, w = softmax(s), o_lat[b][h] = sum_j w_j C_j (fp32, [batch][Hq][r]).
  * Pages selected by several query heads of one KV head are read once.
- * sel / sel_cnt as written by basiskv_route (any ascending, duplicate-free
- * list of valid pages is accepted).  workspace as for basiskv_route (the same
- * buffer may be passed to both).  err_flag may not be NULL.
+ * sel / sel_cnt (device): any selection in basiskv_route's layout (each row a
+ * duplicate-free list of pages of its sequence; a page outside the sequence
+ * sets BASISKV_DEVERR_SELECTION and is skipped).  With sel and sel_cnt both
+ * NULL the call attends over the selection the last basiskv_route or
+ * basiskv_route_group call on the same workspace (same cfg, batch and
+ * max_pages) stored there, without rebuilding it; giving only one of them is
+ * BASISKV_ERR_INVALID_ARG.  workspace as for basiskv_route (the same buffer
+ * may be passed to both).  err_flag may not be NULL.
+ * A group's tiles are shared out among the kernel's warps at run time, so
+ * o_lat may differ between calls in the last bits of fp32 (the order of the
+ * softmax sums), never by more than the rounding of those sums.
  */
 BASISKV_API basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,
                                    const void* q, int32_t batch, const int32_t* sel,
@@ -250,20 +267,27 @@ BASISKV_API basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const 
  * counterpart in the paper: it exists for callers that cannot allocate
  * device memory (a plugin whose host engine owns every allocation, code that
  * runs while its stream is captured into a CUDA graph, a fixed memory budget
- * after start-up).  It computes exactly what basiskv_decode_attn computes, with
- * the same arguments minus the workspace, using a scratch array of 16 MiB that
- * the library keeps in device memory on every GPU where it is loaded, for the
- * life of the process.
- *   - Shapes whose scratch (union lists, counts, split partials) exceeds
+ * after start-up).  It computes exactly what basiskv_decode_attn computes for
+ * a given selection, with the same arguments minus the workspace, using a
+ * scratch array of 16 MiB that the library keeps in device memory on every
+ * GPU where it is loaded, for the life of the process.
+ *   - Arguments are checked exactly as basiskv_decode_attn checks them, in the
+ *     same order; sel and sel_cnt may not be NULL (there is no routing
+ *     workspace to take a selection from).
+ *   - Shapes whose scratch (union lists, counters, split partials) exceeds
  *     16 MiB return BASISKV_ERR_WORKSPACE (with a message on stderr) and
  *     launch nothing; use basiskv_decode_attn then.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
- *   - Every call on a device shares the one array.  Calls that may overlap on
- *     the GPU (different streams without ordering) race and corrupt each
- *     other's results; order them.  The array is zero when the library loads
- *     and every call leaves its counters at zero again, so it needs no
- *     clearing.
+ *     (cudaGetSymbolAddress) in the context current then (the device's
+ *     primary context for CUDA runtime callers) and keeps it; make that first
+ *     call before any stream capture.  Calling from another context on the
+ *     same device, or after cudaDeviceReset, is not supported.
+ *   - Every call on a device shares the one array, whatever its shape.  Calls
+ *     that may overlap on the GPU (different streams without ordering) race
+ *     and corrupt each other's results; order them.  Each call writes all the
+ *     scratch it reads (its first kernel zeroes the counters the second one
+ *     uses), so the array needs no clearing, also between calls of different
+ *     shapes.
  */
 BASISKV_API basiskv_status basiskv_decode_attn_noalloc(const basiskv_config* cfg,
                                                        const basiskv_cache* cache, const void* q,

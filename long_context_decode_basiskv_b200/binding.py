@@ -254,13 +254,18 @@ def route_group(cfg: Config, cache: PagedCache, q: torch.Tensor, reduce: int, se
                                      _ptr(err), _stream(stream)), "basiskv_route_group")
 
 
-def decode_attn(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor,
-                sel_cnt: torch.Tensor, o_lat: torch.Tensor, ws: torch.Tensor, err: torch.Tensor,
+def decode_attn(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: Optional[torch.Tensor],
+                sel_cnt: Optional[torch.Tensor], o_lat: torch.Tensor, ws: torch.Tensor, err: torch.Tensor,
                 stream=None):
+    """Attention over the pages in sel / sel_cnt, or (both None) over the selection the
+    last route / route_group call left in the same workspace."""
     B = q.shape[0]
     _need(q, "q", cfg.dtype, (B, cfg.num_q_heads, cfg.head_dim))
-    _need(sel, "sel", torch.int32, (B, cfg.num_q_heads, cfg.top_k + 2))
-    _need(sel_cnt, "sel_cnt", torch.int32, (B, cfg.num_q_heads))
+    if (sel is None) != (sel_cnt is None):
+        raise ValueError("sel and sel_cnt are given together or not at all")
+    if sel is not None:
+        _need(sel, "sel", torch.int32, (B, cfg.num_q_heads, cfg.top_k + 2))
+        _need(sel_cnt, "sel_cnt", torch.int32, (B, cfg.num_q_heads))
     _need(o_lat, "o_lat", torch.float32, (B, cfg.num_q_heads, cfg.rank_v))
     _need(ws, "workspace", torch.uint8)
     _need(err, "err", torch.int32)

@@ -3,6 +3,7 @@
 #include <stdio.h>
 
 #include "kernels.cuh"
+#include "union.cuh"
 
 namespace bkv {
 
@@ -34,47 +35,91 @@ static basiskv_status check_config(const basiskv_config* c) {
   return BASISKV_OK;
 }
 
-static basiskv_status check_cache(const basiskv_config* c, const basiskv_cache* k, bool need_res) {
-  if (!k || !k->k_raw || !k->c_lat || !k->summary || !k->block_table || !k->seq_len)
-    return BASISKV_ERR_INVALID_ARG;
+static basiskv_status check_cache(const basiskv_config* c, const basiskv_cache* k, bool need_res,
+                                  bool need_summary = true) {
+  if (!k || !k->k_raw || !k->c_lat || !k->block_table || !k->seq_len) return BASISKV_ERR_INVALID_ARG;
+  if (need_summary && !k->summary) return BASISKV_ERR_INVALID_ARG;
   if (need_res && !k->r_res) return BASISKV_ERR_INVALID_ARG;
   if (k->num_phys_pages <= 0 || k->max_pages <= 0) return BASISKV_ERR_INVALID_ARG;
-  if (k->max_pages > kMaxPagesLimit) return BASISKV_ERR_UNSUPPORTED;
-  if (!aligned16(k->k_raw) || !aligned16(k->c_lat) || !aligned16(k->summary) ||
+  if (k->max_pages > kMaxPagesLimit || k->num_phys_pages > kMaxPhysPages) return BASISKV_ERR_UNSUPPORTED;
+  if (!aligned16(k->k_raw) || !aligned16(k->c_lat) || (need_summary && !aligned16(k->summary)) ||
       (need_res && !aligned16(k->r_res)))
     return BASISKV_ERR_INVALID_ARG;
   (void)c;
   return BASISKV_OK;
 }
 
-static int num_sms() {
+int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
 }
 
+// Workspace: routing scores, the routing arrival counters, then the decode
+// scratch of decode_plan() (union lists, counters, tile cursors, split results).
 struct Workspace {
-  size_t scores, decode, total;
+  size_t scores, rcnt, decode, total;
   DecodePlan plan;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// routing scores first, then the decode scratch of decode_plan()
 static Workspace layout(const basiskv_config* c, int batch, int max_pages) {
   Workspace w{};
   w.plan = decode_plan(c->num_q_heads, c->num_kv_heads, c->page_size, c->rank_v, c->top_k, batch, max_pages,
                        c->dtype == BASISKV_BF16, c->head_dim, num_sms());
   w.scores = 0;
-  w.decode = up256((size_t)batch * c->num_q_heads * max_pages * 4);
+  w.rcnt = up256((size_t)batch * c->num_q_heads * max_pages * 4);
+  w.decode = w.rcnt + up256((size_t)batch * c->num_kv_heads * 4);
   w.total = w.decode + w.plan.bytes;
   return w;
 }
 
-static basiskv_status cuda_status(cudaError_t e) {
+basiskv_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return BASISKV_OK;
   fprintf(stderr, "basiskv: CUDA error %s\n", cudaGetErrorString(e));
   return BASISKV_ERR_CUDA;
+}
+
+// Validation shared by basiskv_decode_attn and basiskv_decode_attn_noalloc
+// (sel and sel_cnt are both given, or both NULL).
+basiskv_status check_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache, const void* q, int32_t batch,
+                                 const int32_t* sel, const int32_t* sel_cnt, const float* o_lat,
+                                 const int32_t* err_flag) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if ((s = check_cache(cfg, cache, false, false)) != BASISKV_OK) return s;
+  if (batch < 0) return BASISKV_ERR_INVALID_ARG;
+  if (batch == 0) return BASISKV_OK;
+  if (!q || !o_lat || !err_flag || (!sel) != (!sel_cnt)) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(q)) return BASISKV_ERR_INVALID_ARG;
+  return BASISKV_OK;
+}
+
+DecodePlan plan_decode_attn(const basiskv_config* cfg, int32_t batch, int32_t max_pages) {
+  return decode_plan(cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v, cfg->top_k, batch, max_pages,
+                     cfg->dtype == BASISKV_BF16, cfg->head_dim, num_sms());
+}
+
+// Union lists from sel (when given), then the attention kernel, into `scratch`
+// laid out by `plan`.
+basiskv_status run_decode_attn(const DecodePlan& plan, const basiskv_config* cfg, const basiskv_cache* cache,
+                               const void* q, int32_t batch, const int32_t* sel, const int32_t* sel_cnt,
+                               float* o_lat, char* scratch, int32_t* err_flag, void* stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  if (sel) {
+    const UnionParams u{sel, sel_cnt, cache->block_table, cache->seq_len,
+                        reinterpret_cast<uint32_t*>(scratch + plan.list_off),
+                        reinterpret_cast<uint32_t*>(scratch + plan.ucount_off),
+                        reinterpret_cast<int32_t*>(scratch + plan.cnt_off), err_flag, cfg->num_q_heads,
+                        cfg->num_kv_heads, cfg->page_size, cache->max_pages, cache->num_phys_pages, cfg->top_k,
+                        plan.ustride};
+    cudaError_t e = launch_union(u, batch, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  DecodeArgs a{q, cache->k_raw, cache->c_lat, o_lat, err_flag, cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim,
+               cfg->page_size, cfg->rank_v, cache->num_phys_pages, cfg->dtype == BASISKV_BF16};
+  return cuda_status(launch_decode_attn(plan, a, scratch, batch, st));
 }
 
 }  // namespace bkv
@@ -159,9 +204,13 @@ static basiskv_status route_common(const basiskv_config* cfg, const basiskv_cach
   if (!ws || ws_bytes < w.total || !aligned16(ws)) return BASISKV_ERR_WORKSPACE;
   char* wsb = static_cast<char*>(ws);
   float* sc = scores ? scores : reinterpret_cast<float*>(wsb + w.scores);
+  uint32_t* lists = reinterpret_cast<uint32_t*>(wsb + w.decode + w.plan.list_off);
+  int32_t* acnt = reinterpret_cast<int32_t*>(wsb + w.decode + w.plan.cnt_off);
   RouteParams rp{q, cache->summary, cache->block_table, cache->seq_len, sc, sel, sel_cnt, err_flag,
                  batch, cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cache->max_pages,
-                 cache->num_phys_pages, cfg->top_k, scores ? 1 : 0, group_mode};
+                 cache->num_phys_pages, cfg->top_k, scores ? 1 : 0, group_mode,
+                 lists, reinterpret_cast<uint32_t*>(wsb + w.decode + w.plan.ucount_off),
+                 reinterpret_cast<int32_t*>(wsb + w.rcnt), acnt, w.plan.ustride};
   return cuda_status(launch_route(rp, cfg->head_dim, cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream));
 }
 
@@ -182,18 +231,12 @@ basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cach
                                    const void* q, int32_t batch, const int32_t* sel,
                                    const int32_t* sel_cnt, float* o_lat, void* ws, size_t ws_bytes,
                                    int32_t* err_flag, void* stream) {
-  basiskv_status s = check_config(cfg);
-  if (s != BASISKV_OK) return s;
-  if ((s = check_cache(cfg, cache, false)) != BASISKV_OK) return s;
-  if (batch == 0) return BASISKV_OK;
-  if (!q || !sel || !sel_cnt || !o_lat || !err_flag || batch < 0) return BASISKV_ERR_INVALID_ARG;
-  if (!aligned16(q)) return BASISKV_ERR_INVALID_ARG;
+  basiskv_status s = check_decode_attn(cfg, cache, q, batch, sel, sel_cnt, o_lat, err_flag);
+  if (s != BASISKV_OK || batch == 0) return s;
   const Workspace w = layout(cfg, batch, cache->max_pages);
   if (!ws || ws_bytes < w.total || !aligned16(ws)) return BASISKV_ERR_WORKSPACE;
-  DecodeArgs a{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, sel, sel_cnt, o_lat, err_flag,
-               cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->page_size, cfg->rank_v,
-               cache->max_pages, cache->num_phys_pages, cfg->top_k, cfg->dtype == BASISKV_BF16};
-  return cuda_status(launch_decode_attn(w.plan, a, static_cast<char*>(ws) + w.decode, batch, (cudaStream_t)stream));
+  return run_decode_attn(w.plan, cfg, cache, q, batch, sel, sel_cnt, o_lat, static_cast<char*>(ws) + w.decode,
+                         err_flag, stream);
 }
 
 basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors* f, const float* o_lat,

@@ -7,176 +7,198 @@
 // restricted to the selected tokens, with the weights applied to the rank-r
 // Value latents instead of full-width values.
 //
-// One launch: one CTA per (sequence, KV head, split of the union); the splits
-// fill one resident wave (decode_plan).  Each CTA first merges the G query
-// heads' selections into the ascending union of pages with a G-bit head mask
-// per page (a page chosen by several heads of a group is read once) and keeps
-// its split's equal share of it.  Two kernels stream the slice's 16-token
-// tiles (raw K rows and C rows, each contiguous in the page block) with 1-D
-// bulk copies (cp.async.bulk, mbarrier completion, bounded waits, no
-// multicast):
-//   * attn_mma_kernel (bf16, the main path): four warps per CTA, each with its
-//     own 3-slot ring, run all G heads of the group on the tensor cores
-//     (mma.sync m16n8k16: scores with heads as rows, online softmax in base
-//     2, P.C accumulated in registers); see the section below.
-//   * attn_kernel (fp32 and shapes without the swizzled layout): warp 0
-//     produces into a shared ring, warps 1..G consume, one per query head of
-//     the group, forming 16 exact scores per tile on the CUDA cores.
-// Each head's split result (max, sum, acc[r]) goes to the workspace; the last
-// CTA of a group to finish (counted with an atomic) merges the group's splits
-// with the log-sum-exp rule and writes o_lat.
+// The pages of a (sequence, KV head) group come as a union list (union.cuh):
+// every page chosen by any of the group's G query heads, once, with a head
+// mask and its physical id resolved.  The routing kernel writes the lists;
+// when the caller passes its own selection, union_kernel builds them from it.
+// One launch then streams the lists, the splits filling one resident wave
+// (decode_plan).  Each split's result per
+// head (max, sum, acc[r]) goes to scratch; the last CTA of a group to finish
+// (counted with an atomic) merges the group's splits with the log-sum-exp rule
+// and writes o_lat.  Two kernels:
+//   * attn_mma_kernel (bf16 with the swizzled K/C layout, the main path): the
+//     groups' 16-token tiles, laid end to end, are cut into equal contiguous
+//     runs, one per CTA, so every SM streams the same bytes whatever the
+//     union sizes (a CTA's run may cross group boundaries; it closes each
+//     group it leaves).  Four warps per CTA take the run's tiles round-robin,
+//     each with its own ring of bulk copies (cp.async.bulk, mbarrier
+//     completion, bounded waits, no multicast), and run all G heads of the
+//     group on the tensor cores (mma.sync m16n8k16).  The split of the work
+//     depends only on the union sizes, so the output is reproducible.
+//   * attn_kernel (fp32 and shapes without the swizzled layout): each split
+//     takes an equal share of the list; warp 0 produces into a shared ring,
+//     warps 1..G consume, one per query head, on the CUDA cores.
 // HBM-bound: every byte of the union's pages is read once.
 #include "kernels.cuh"
+#include "union.cuh"
 
 namespace bkv {
 
 constexpr int kTile = 16;           // tokens per tile
-constexpr int kStages = 4;          // ring depth per CTA
-constexpr int kCoreCtasPerSm = 6;   // resident CTAs per SM of the CUDA-core attention kernel
-constexpr int kMmaCtasPerSm = 3;    // ... and of the tensor-core one (registers and shared memory)
+constexpr int kStages = 4;          // ring depth per CTA of the CUDA-core kernel
+constexpr int kCoreCtasMax = 6;     // resident CTAs per SM of the CUDA-core attention kernel, at most
+constexpr int kMmaCtasPerSm = 3;    // ... and of the tensor-core one (registers)
+constexpr int kMmaWarps = 4;        // warps per CTA of the tensor-core kernel
+constexpr int kMinWarpTiles = 2;    // tiles per warp of the tensor-core kernel, at least
+constexpr int kMinSplitTiles = 8;   // tiles per split of the CUDA-core kernel (full unions), at least
+constexpr size_t kSmemPerSm = 228 * 1024;
+constexpr size_t kSmemPerCtaReserved = 1024;
+
+static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// shared memory of the tensor-core kernel: rings, their barriers, one group's result
+static size_t mma_smem_bytes(int d, int r, int slots, int G) {
+  const size_t stage = ((size_t)kTile * (d + r) * 2 + 127) & ~(size_t)127;
+  return (size_t)kMmaWarps * slots * (stage + 8) + (size_t)G * (r + 2) * 4;
+}
+// ... and of the CUDA-core kernel: ring and full / empty barriers
+static size_t core_smem_bytes(int d, int r, int esize) {
+  const size_t stage = ((size_t)kTile * (d + r) * esize + 127) & ~(size_t)127;
+  return (size_t)kStages * stage + 2 * kStages * 8;
+}
 
 // ---------------------------------------------------------------------------
 // plan: splits per (sequence, KV head) and the scratch layout
 // ---------------------------------------------------------------------------
-static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-// The splits fill one resident wave of the kernel exactly: with q = slots /
-// groups and m = slots % groups, the last m groups get q + 1 splits and the
-// others q (at least one each), so every SM holds the same number of CTAs and
-// about the same number of tiles (the memory system gives every SM a similar
-// share of the bandwidth, so an SM with more work would finish last).  Each
-// split takes an equal share of its group's union at run time.  The first
-// groups' unused CTAs (split q) exit at once and free their slots.
+// Tensor-core kernel: the grid is one resident wave; each CTA takes an equal
+// run of the groups' tiles laid end to end and writes one partial result per
+// group its run touches, in slot CTA + group (so grid + groups slots).
+// CUDA-core kernel: one CTA per group at least, up to one resident wave; the
+// CTAs past one per group are shared out among the groups in proportion to
+// their tiles when the kernel runs (assign_cta), each split keeping at least
+// kMinSplitTiles tiles of a full union.  Each CTA writes one partial result.
 DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d,
                        int num_sms) {
   DecodePlan pl{};
-  const long long slots = (long long)num_sms * (kc_swizzled(bf16, d, r) ? kMmaCtasPerSm : kCoreCtasPerSm);
   const int G = Hq / Hkv;
   long long um = (long long)G * (top_k + 2);
   if (um > max_pages) um = max_pages;
   pl.umax = (int)um;
   pl.tpp = page / kTile;
+  pl.ustride = union_stride_words(pl.umax);
+  int per_sm;
+  if (kc_swizzled(bf16, d, r)) {
+    // three slots per warp where three CTAs fit, else two
+    pl.ring_slots = 3;
+    if (kMmaCtasPerSm * (mma_smem_bytes(d, r, 3, G) + kSmemPerCtaReserved) > kSmemPerSm) pl.ring_slots = 2;
+    per_sm = (int)(kSmemPerSm / (mma_smem_bytes(d, r, pl.ring_slots, G) + kSmemPerCtaReserved));
+    if (per_sm > kMmaCtasPerSm) per_sm = kMmaCtasPerSm;
+  } else {
+    pl.ring_slots = 0;
+    per_sm = (int)(kSmemPerSm / (core_smem_bytes(d, r, bf16 ? 2 : 4) + kSmemPerCtaReserved));
+    if (per_sm > kCoreCtasMax) per_sm = kCoreCtasMax;
+  }
+  if (per_sm < 1) per_sm = 1;
+  const long long slots = (long long)num_sms * per_sm;
   const long long groups = (long long)batch * Hkv;
-  long long q = slots / groups, m = slots % groups;
-  if (q >= pl.umax) {
-    q = pl.umax;
-    m = 0;
+  if (pl.ring_slots > 0) {
+    pl.grid = (int)slots;
+    pl.extra = 0;
+  } else {
+    long long per_group = ((long long)pl.umax * pl.tpp + kMinSplitTiles - 1) / kMinSplitTiles;
+    if (per_group < 1) per_group = 1;
+    long long grid = slots < groups * per_group ? slots : groups * per_group;
+    if (grid < groups) grid = groups;
+    pl.grid = (int)grid;
+    pl.extra = (int)(grid - groups);
   }
-  if (q < 1) {
-    q = 1;
-    m = 0;
-  }
-  pl.nsplit_lo = (int)q;
-  pl.nsplit = (int)(m > 0 ? q + 1 : q);
-  pl.rich_from = (int)(groups - m);
-  pl.eps = (pl.umax + pl.nsplit_lo - 1) / pl.nsplit_lo;
   size_t off = 0;
+  pl.list_off = off;
+  off += up256((size_t)batch * Hkv * pl.ustride * 4);
+  pl.ucount_off = off;
+  off += up256((size_t)batch * Hkv * 4);
   pl.cnt_off = off;
   off += up256((size_t)batch * Hkv * 4);
   pl.part_off = off;
-  off += up256((size_t)batch * Hq * pl.nsplit * (r + 2) * 4);
+  off += up256((size_t)(pl.grid + groups) * G * (r + 2) * 4);
   pl.bytes = off;
   return pl;
 }
 
-// ---------------------------------------------------------------------------
-// union of the group's selections, built by every CTA for its own split
-// ---------------------------------------------------------------------------
-// All threads of the CTA call this.  It merges the G heads' selections of
-// (b, g) into per-page head masks in `words` (shared scratch of at least
-// ceil(max_pages / 4) words) and ranks the selected pages in ascending order
-// with a block scan.  The union of U pages is cut into nsplit equal slices of
-// ceil(U / nsplit) entries; the entries of slice `split` are stored as
-// page | mask << 24 in `ent` (shared).  Every load of the selections is issued
-// before the first barrier, so their latencies overlap.
-struct UnionSlice {
-  int U;       // union size of (b, g)
-  int e0;      // first union entry of this split
-  int cnt;     // entries in this split (0: no work)
-  int active;  // splits of (b, g) with work
-};
-constexpr int kUnionLoads = 8;  // selection entries a thread loads before the first barrier
-
-__device__ UnionSlice union_slice(const AttnParams& p, int b, int g, int G, int split, uint32_t* words,
-                                  uint32_t* ent, int* warp_tot, int* s_cnt) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int row_len = p.top_k + 2;
-  const size_t row0 = (size_t)b * p.Hq + (size_t)g * G;
-  const int total = G * row_len;
-  const int32_t* selg = p.sel + row0 * row_len;  // the G rows are contiguous
-  const int L = p.seq_len[b];
-  if (tid < G) s_cnt[tid] = min(p.sel_cnt[row0 + tid], row_len);
-  int v[kUnionLoads];
-#pragma unroll
-  for (int j = 0; j < kUnionLoads; ++j) {
-    const int i = tid + j * nthr;
-    v[j] = (i < total) ? selg[i] : -1;
-  }
-  for (int i = tid; i < (p.max_pages + 3) / 4; i += nthr) words[i] = 0u;
-  __syncthreads();
-  const int n = max(0, min((L + p.page - 1) / p.page, p.max_pages));
-  auto mark = [&](int i, int pg) {
-    const int hi = i / row_len;
-    if (i - hi * row_len >= s_cnt[hi]) return;
-    if (pg < 0 || pg >= n) {
-      set_err(p.err, BASISKV_DEVERR_SELECTION);
-      return;
+// Which group CTA c works on.  Group g (in b * Hkv + g order) has t_g = U_g *
+// tpp tiles, P_g tiles before it and T in all; it gets the CTAs [c_g,
+// c_{g+1}) with c_g = g + floor(extra * P_g / T): at least one, the rest in
+// proportion to its tiles, grid = groups + extra CTAs in all.  All threads call
+// this (each scans a contiguous run of groups, read twice from L2); the result
+// lands in s_asg[4] = {group, split, splits, first CTA of the group}.
+__device__ __forceinline__ void assign_cta(const AttnParams& p, int c, int* warp_tot, int* s_asg) {
+  const int tid = threadIdx.x, nthr = blockDim.x, NG = p.ngroups;
+  auto tiles = [&](int g) { return (int)min(__ldcg(p.ucount + g), (uint32_t)p.umax) * p.tpp; };
+  const int per = (NG + nthr - 1) / nthr;
+  const int g0 = min(NG, tid * per), g1 = min(NG, g0 + per);
+  int local = 0;
+  for (int g = g0; g < g1; ++g) local += tiles(g);
+  int T;
+  long long P = block_exclusive_scan(local, warp_tot, T);
+  for (int g = g0; g < g1; ++g) {
+    const long long pn = P + tiles(g);
+    const int cg = g + (int)(T > 0 ? ((long long)p.extra * P) / T : 0);
+    const int cn = g + 1 + (int)(T > 0 ? ((long long)p.extra * pn) / T : (g + 1 == NG ? p.extra : 0));
+    if (c >= cg && c < cn) {
+      s_asg[0] = g;
+      s_asg[1] = c - cg;
+      s_asg[2] = cn - cg;
+      s_asg[3] = cg;
     }
-    atomicOr(&words[pg >> 2], (1u << hi) << ((pg & 3) * 8));
-  };
-#pragma unroll
-  for (int j = 0; j < kUnionLoads; ++j) {
-    const int i = tid + j * nthr;
-    if (i < total) mark(i, v[j]);
-  }
-  for (int i = tid + kUnionLoads * nthr; i < total; i += nthr) mark(i, selg[i]);
-  __syncthreads();
-  const int per = (n + nthr - 1) / nthr;
-  const int lo = tid * per, hi = min(n, lo + per);
-  int c = 0;
-  for (int pg = lo; pg < hi; ++pg) c += ((words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu) ? 1 : 0;
-  int tot;
-  int pos = block_exclusive_scan(c, warp_tot, tot);
-  UnionSlice sl;
-  sl.U = tot;
-  const int ns = ((int)(b * p.Hkv + g) >= p.rich_from) ? p.nsplit : p.nsplit_lo;  // splits of this group
-  const int eps = (tot + ns - 1) / ns;
-  sl.e0 = split * eps;
-  sl.cnt = (split < ns) ? max(0, min(tot, sl.e0 + eps) - sl.e0) : 0;
-  sl.active = eps > 0 ? (tot + eps - 1) / eps : 0;
-  for (int pg = lo; pg < hi && pos < sl.e0 + sl.cnt; ++pg) {
-    const uint32_t m = (words[pg >> 2] >> ((pg & 3) * 8)) & 0xffu;
-    if (m) {
-      if (pos >= sl.e0) ent[pos - sl.e0] = (uint32_t)pg | (m << 24);
-      ++pos;
-    }
+    P = pn;
   }
   __syncthreads();
-  return sl;
 }
 
-// Offset of the split's entry list in dynamic shared memory: after the ring
-// (and its barriers), and after the page-mask scratch of union_slice.
-__host__ __device__ __forceinline__ size_t attn_ent_offset(size_t ring_bytes, int max_pages) {
-  const size_t masks = ((size_t)max_pages + 15) & ~(size_t)15;
-  return ((ring_bytes > masks ? ring_bytes : masks) + 15) & ~(size_t)15;
+// ---------------------------------------------------------------------------
+// union lists from a given selection
+// ---------------------------------------------------------------------------
+// One CTA per (KV head, sequence): the G heads' selections are OR-ed into one
+// byte of head bits per page (shared memory), then write_union_list stores the
+// ascending list.  A selected page outside [0, n) sets
+// BASISKV_DEVERR_SELECTION and is dropped.
+constexpr int kUnionThreads = 256;
+
+__global__ void __launch_bounds__(kUnionThreads) union_kernel(UnionParams u) {
+  extern __shared__ __align__(16) uint32_t masks[];  // ceil(max_pages / 4) words
+  __shared__ int warp_tot[32];
+  grid_dep_wait();      // the selection may come from the kernel before this one
+  allow_dependents();   // the attention kernel may launch; it waits for this grid
+  const int g = blockIdx.x, b = blockIdx.y;
+  union_from_selection(u.sel, u.sel_cnt, u.block_table, u.seq_len[b], b, g, u.Hq, u.Hkv, u.page, u.max_pages,
+                       u.num_phys, u.top_k, u.lists + ((size_t)b * u.Hkv + g) * u.ustride,
+                       u.ucount + (size_t)b * u.Hkv + g, u.acnt, u.err, masks, nullptr, warp_tot);
+}
+
+cudaError_t launch_union(const UnionParams& u, int batch, cudaStream_t st) {
+  const size_t smem = (size_t)((u.max_pages + 3) / 4) * 4;
+  cudaError_t e = ensure_smem((const void*)union_kernel, smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(u.Hkv, batch);
+  cfg.blockDim = dim3(kUnionThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, union_kernel, u);
 }
 
 // After writing its split results, a CTA counts itself on the group's counter;
-// the last one of the group merges.  The merging CTA puts the counter back to
-// zero, so counters are zero between calls (the workspace is zero-filled once).
+// the last one of the group merges.  The merging CTA puts the counter (and the
+// group's tile cursor) back to zero, so both are zero between calls.
+// The barrier orders every thread's split results before thread 0's release
+// fence and atomic; the last CTA's thread 0 fences again (acquire) before the
+// barrier that lets its threads read the other CTAs' results.
 __device__ __forceinline__ bool last_of_group(const AttnParams& p, size_t bg, int nsplit_active, int* s_last) {
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const int prev = atomicAdd(&p.cnt[bg], 1);
     if (prev >= nsplit_active) set_err(p.err, BASISKV_DEVERR_WORKSPACE);
     *s_last = (prev == nsplit_active - 1);
+    if (*s_last) __threadfence();
   }
   __syncthreads();
-  if (!*s_last) return false;
-  __threadfence();
-  return true;
+  return *s_last != 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -219,51 +241,55 @@ __device__ __forceinline__ void load_pair(const T* row, int dim, float& a, float
 }
 
 // The last CTA of a (sequence, KV head) group merges the group's split
-// results: for each of its G heads, log-sum-exp over the splits.  Heads are
-// spread over `nw` warps starting at warp index `wi`.
-__device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, int g, int G, int r,
-                                                   int nsplit_active, int wi, int nw, int lane) {
+// results: for each of its G heads, log-sum-exp over the splits, whose
+// partials sit in the slots of the group's CTAs (slot0 .. slot0 + ns - 1).
+// Heads are spread over `nw` warps starting at warp index `wi`; a warp issues
+// the loads of up to eight splits (max, sum and its lanes' dimensions) before
+// it uses any.
+__device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, int g, int G, int r, int slot0,
+                                                   int ns, int wi, int nw, int lane) {
   constexpr int kDimIt = 4;  // r <= 128: dims lane + 32 k
   constexpr int kBatch = 8;  // splits whose values are loaded together
   const int stride = r + 2;
   for (int hi = wi; hi < G; hi += nw) {
     const int h = g * G + hi;
-    const float* base = p.part + ((size_t)b * p.Hq + h) * p.nsplit * stride;
-    float M = -INFINITY;
-    for (int s = lane; s < nsplit_active; s += 32) M = fmaxf(M, __ldcg(base + (size_t)s * stride));
-    M = warp_max(M);
-    float Ls = 0.f;
+    const float* base = p.part + ((size_t)slot0 * G + hi) * stride;
+    const size_t sstride = (size_t)G * stride;  // between consecutive CTAs' slots
+    float M = -INFINITY, Ls = 0.f;
     float acc[kDimIt] = {0.f, 0.f, 0.f, 0.f};
-    for (int c0 = 0; c0 < nsplit_active; c0 += 32) {
-      // lane s: the weight of split c0 + s
-      const int sl = c0 + lane;
-      float wl = 0.f;
-      if (sl < nsplit_active) {
-        const float ms = __ldcg(base + (size_t)sl * stride);
-        if (ms != -INFINITY) {
-          wl = exp2f(ms - M);
-          Ls += __ldcg(base + (size_t)sl * stride + 1) * wl;
-        }
+    for (int s0 = 0; s0 < ns; s0 += kBatch) {
+      const int cn = min(kBatch, ns - s0);
+      // lane j < cn: max and sum of split s0 + j; every lane: its dims of every split
+      float mj = -INFINITY, lj = 0.f;
+      if (lane < cn) {
+        mj = __ldcg(base + (size_t)(s0 + lane) * sstride);
+        lj = __ldcg(base + (size_t)(s0 + lane) * sstride + 1);
       }
-      const int cn = min(32, nsplit_active - c0);
-      for (int j0 = 0; j0 < cn; j0 += kBatch) {
-        float x[kBatch][kDimIt];
+      float x[kBatch][kDimIt];
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j)
+      for (int j = 0; j < kBatch; ++j)
 #pragma unroll
-          for (int k = 0; k < kDimIt; ++k) {
-            const int dim = lane + 32 * k;
-            x[j][k] = (j0 + j < cn && dim < r) ? __ldcg(base + (size_t)(c0 + j0 + j) * stride + 2 + dim) : 0.f;
-          }
+        for (int k = 0; k < kDimIt; ++k) {
+          const int dim = lane + 32 * k;
+          x[j][k] = (j < cn && dim < r) ? __ldcg(base + (size_t)(s0 + j) * sstride + 2 + dim) : 0.f;
+        }
+      const float Mn = fmaxf(M, warp_max(mj));
+      if (Mn != -INFINITY) {
+        const float cf = (M == -INFINITY) ? 0.f : exp2f(M - Mn);  // rescale what the earlier batches summed
+        Ls *= cf;
+#pragma unroll
+        for (int k = 0; k < kDimIt; ++k) acc[k] *= cf;
+        const float wl = (mj == -INFINITY) ? 0.f : exp2f(mj - Mn);
+        Ls += warp_sum(lj * wl);
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
-          const float wt = __shfl_sync(kFull, wl, (j0 + j) & 31);
+          const float wt = __shfl_sync(kFull, wl, j);
 #pragma unroll
           for (int k = 0; k < kDimIt; ++k) acc[k] = fmaf(x[j][k], wt, acc[k]);
         }
+        M = Mn;
       }
     }
-    Ls = warp_sum(Ls);
 #pragma unroll
     for (int k = 0; k < kDimIt; ++k) {
       const int dim = lane + 32 * k;
@@ -272,92 +298,97 @@ __device__ __forceinline__ void merge_group_splits(const AttnParams& p, int b, i
   }
 }
 
+// Wait (bounded) for the bulk copies a timed-out ring may still have in flight:
+// the full barrier of every tile in [from, to) in a ring of `slots` stages.
+// Returns false if one of them also gives up.
+__device__ __forceinline__ bool drain_ring(uint64_t* full, int slots, int from, int to) {
+  bool ok = true;
+  for (int t = from; t < to; ++t) ok = mbar_wait_bounded(&full[t % slots], (uint32_t)((t / slots) & 1)) && ok;
+  return ok;
+}
+
 template <typename T, int D, int G, int CU>
 __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   constexpr int DPL = D / 32;
-  allow_dependents();  // the out-projection may launch and start streaming its weights
-  grid_dep_wait();     // the selection is complete (this kernel may launch before it ends)
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint32_t meta[kStages];  // head mask | valid tokens << 8 of the tile in each stage
-  __shared__ int s_last;
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  __shared__ int s_last, s_fail, s_issued, s_consumed;
+  __shared__ int warp_tot[32];
+  __shared__ int s_asg[4];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.r;
-  const size_t bg = (size_t)b * p.Hkv + g;
   const uint32_t k_bytes = kTile * D * sizeof(T);
   const uint32_t c_bytes = kTile * r * sizeof(T);
   const uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
-  // shared memory: [ring | barriers] (page-mask scratch while the union is built) then the split's entries
-  uint32_t* ent = reinterpret_cast<uint32_t*>(smem + attn_ent_offset(kStages * stage_bytes + 2 * kStages * 8, p.max_pages));
-  __shared__ int warp_tot[32];
-  __shared__ int s_cnt[8];
-  const UnionSlice sl = union_slice(p, b, g, G, split, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
-  const int U = sl.U, nsplit_active = sl.active;
-  if (sl.cnt == 0) {
-    // no work in this split; split 0 of an empty group still defines its output
-    if (split == 0 && U == 0)
-      for (int i = threadIdx.x; i < G * r; i += blockDim.x)
-        p.o_lat[((size_t)b * p.Hq + (size_t)g * G) * r + i] = 0.f;
-    return;
-  }
-  const int nent = sl.cnt;
-  const int ntiles = nent * p.tpp;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * stage_bytes);
   uint64_t* empty = full + kStages;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], G);
     }
     fence_mbar_init();
+    s_fail = 0;
+    s_issued = 0;
+    s_consumed = 0;
   }
   __syncthreads();
+  grid_dep_wait();     // the union lists are complete (this kernel may launch before their writer ends)
+  allow_dependents();  // the out-projection may launch and start streaming its weights
+  assign_cta(p, blockIdx.x, warp_tot, s_asg);
+  const int bg = s_asg[0], split = s_asg[1], ns = s_asg[2], slot0 = s_asg[3];
+  const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+  // the query row of a consumer warp
+  float qf[DPL];
+  if (warp >= 1) {
+    const T* qr = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G + warp - 1) * D + lane * DPL;
+#pragma unroll
+    for (int u = 0; u < DPL; ++u) qf[u] = Elem<T>::to_f(qr[u]) * p.qscale;
+  }
+
+  const uint32_t* list = p.lists + (size_t)bg * p.ustride;
+  const int U = min((int)__ldcg(list), p.umax);
+  const int tail_valid = (int)__ldcg(list + 1);
+  const int eps = (U + ns - 1) / ns;
+  const int e0 = split * eps;
+  const int nent = max(0, min(U, e0 + eps) - e0);
+  const int ntiles = nent * p.tpp;
 
   bool ok = true;
   if (warp == 0) {
     // ---------------- producer ----------------
-    const int L = p.seq_len[b];
-    const int n = min((L + p.page - 1) / p.page, p.max_pages);
-    const int last_valid = L - (n - 1) * p.page;
     const T* kbase = static_cast<const T*>(p.k_raw);
     const T* cbase = static_cast<const T*>(p.c_lat);
+    int t = 0;
     for (int cb = 0; cb < nent && ok; cb += 32) {
-      // lane e holds entry cb + e of this split
-      uint32_t my_mask = 0;
-      int my_phys = -1, my_valid = 0;
+      // lane e holds entry e0 + cb + e of the list
+      uint32_t my_en = kNoPage;
+      int my_valid = 0;
       if (cb + lane < nent) {
-        const uint32_t en = ent[cb + lane];
-        const int pg = (int)(en & 0xffffffu);
-        my_mask = en >> 24;
-        if (pg < n) {
-          const int ph = p.block_table[(size_t)b * p.max_pages + pg];
-          if (ph >= 0 && ph < p.num_phys) {
-            my_phys = ph;
-            my_valid = (pg == n - 1) ? last_valid : p.page;
-          } else {
-            set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
-          }
-        }
+        const int e = e0 + cb + lane;
+        my_en = __ldcg(list + 4 + e);
+        my_valid = (e == U - 1) ? tail_valid : p.page;
       }
       const int t_end = min(nent, cb + 32) * p.tpp;
-      for (int t = cb * p.tpp; t < t_end; ++t) {
+      for (; t < t_end; ++t) {
         const int el = t / p.tpp - cb, sub = t - (t / p.tpp) * p.tpp;
-        const int ph = __shfl_sync(kFull, my_phys, el);
-        const uint32_t mask = __shfl_sync(kFull, my_mask, el);
+        const uint32_t en = __shfl_sync(kFull, my_en, el);
         const int pv = __shfl_sync(kFull, my_valid, el);
-        const int valid = (ph >= 0) ? min(kTile, max(0, pv - sub * kTile)) : 0;
+        const uint32_t id = en & kNoPage;
+        if (lane == 0 && id != kNoPage && id >= (uint32_t)p.num_phys) set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
+        const int valid = (id < (uint32_t)p.num_phys) ? min(kTile, max(0, pv - sub * kTile)) : 0;
         const int s = t % kStages;
-        if (t >= kStages && !mbar_wait_bounded(&empty[s], (uint32_t)(((t / kStages) - 1) & 1))) {
+        // every lane waits; the warp gives up together if any lane's wait expired
+        if (t >= kStages && !__all_sync(kFull, mbar_wait_bounded(&empty[s], (uint32_t)(((t / kStages) - 1) & 1)))) {
           ok = false;
           break;
         }
         if (lane == 0) {
-          meta[s] = mask | ((uint32_t)valid << 8);
+          meta[s] = (en >> 24) | ((uint32_t)valid << 8);
           unsigned char* st = smem + (size_t)s * stage_bytes;
           fence_proxy_async_smem();
           if (valid > 0) {
-            const size_t row0 = ((size_t)ph * p.Hkv + g) * p.page + (size_t)sub * kTile;
+            const size_t row0 = ((size_t)id * p.Hkv + g) * p.page + (size_t)sub * kTile;
             mbar_arrive_expect_tx(&full[s], k_bytes + c_bytes);
             bulk_g2s(st, kbase + row0 * D, k_bytes, &full[s]);
             bulk_g2s(st + k_bytes, cbase + row0 * r, c_bytes, &full[s]);
@@ -368,23 +399,19 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
         __syncwarp();
       }
     }
+    if (lane == 0) s_issued = t;
   } else {
     // ---------------- consumer: one query head ----------------
     const int hi = warp - 1;
     const int h = g * G + hi;
-    float qf[DPL];
-    {
-      const T* qr = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D + lane * DPL;
-#pragma unroll
-      for (int u = 0; u < DPL; ++u) qf[u] = Elem<T>::to_f(qr[u]) * p.qscale;
-    }
     float m_run = -INFINITY, l_run = 0.f;
     float acc[CU][2];
 #pragma unroll
     for (int u = 0; u < CU; ++u) acc[u][0] = acc[u][1] = 0.f;
-    for (int t = 0; t < ntiles; ++t) {
+    int t = 0;
+    for (; t < ntiles; ++t) {
       const int s = t % kStages;
-      if (!mbar_wait_bounded(&full[s], (uint32_t)((t / kStages) & 1))) {
+      if (!__all_sync(kFull, mbar_wait_bounded(&full[s], (uint32_t)((t / kStages) & 1)))) {
         ok = false;
         break;
       }
@@ -438,9 +465,10 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
+    if (lane == 0) atomicMax(&s_consumed, t);
     // this head's result for the split
     const float lsum = warp_sum(l_run);
-    float* out = p.part + (((size_t)b * p.Hq + h) * p.nsplit + split) * (r + 2);
+    float* out = p.part + ((size_t)blockIdx.x * G + hi) * (r + 2);
     if (lane == 0) {
       out[0] = m_run;
       out[1] = lsum;
@@ -454,11 +482,25 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
       }
     }
   }
-  if (!ok) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
+  if (!ok) s_fail = 1;
+  __syncthreads();
+  if (s_fail) {
+    // a wait gave up: let the copies still in flight land before the CTA's
+    // shared memory is released, and mark the split's result
+    if (threadIdx.x == 0) {
+      set_err(p.err, BASISKV_DEVERR_TIMEOUT);
+      drain_ring(full, kStages, s_consumed, s_issued);
+    }
+    if (warp >= 1 && lane == 0) {
+      float* out = p.part + ((size_t)blockIdx.x * G + warp - 1) * (r + 2);
+      out[0] = 0.f;                          // the merge weighs this split's sum ...
+      out[1] = __int_as_float(0x7fc00000);   // ... which is NaN: the head's output becomes NaN
+    }
+  }
 
   // the last CTA of the group to finish merges every split of its G heads
-  if (!last_of_group(p, bg, nsplit_active, &s_last)) return;
-  if (warp >= 1) merge_group_splits(p, b, g, G, r, nsplit_active, warp - 1, G, lane);
+  if (!last_of_group(p, bg, ns, &s_last)) return;
+  if (warp >= 1) merge_group_splits(p, b, g, G, r, slot0, ns, warp - 1, G, lane);
   if (threadIdx.x == 0) p.cnt[bg] = 0;
 }
 
@@ -471,9 +513,6 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
 // A fragments line up), rounded to bf16.  K and C rows are XOR-swizzled in the
 // page (see swz()), so ldmatrix reads 8 rows without bank conflicts.
 // ---------------------------------------------------------------------------
-constexpr int kMmaWarps = 4;       // warps per CTA; each streams and consumes its own tiles
-constexpr int kMmaWarpStages = 3;  // ring slots per warp
-
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -496,94 +535,144 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int D, int G, int NT>
-__global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams p) {
+// Work of the tensor-core kernel: the groups' tiles laid end to end (b * Hkv
+// + g order, T in all) and cut into contiguous runs of q = ceil(T / C) tiles,
+// run c for CTA c.  Every CTA but the last ones streams the same number of
+// tiles however the union sizes of the groups differ (no split has more than
+// the least possible maximum), and the CTAs holding a group's tiles are
+// consecutive, each with at least one of them.
+// q is rounded up to whole rounds of the CTA's warps (the slowest warp sets the
+// CTA's time, so this costs nothing) and to kMinWarpTiles tiles per warp.
+__device__ __forceinline__ int run_length(int T, int C) {
+  const int per_warp = (T + kMmaWarps * C - 1) / (kMmaWarps * C);
+  return kMmaWarps * max(per_warp, kMinWarpTiles);
+}
+
+template <int D, int G, int NT, int SW>
+__global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel(AttnParams p) {
   constexpr int KS = D / 16;
-  allow_dependents();  // the out-projection may launch and start streaming its weights
-  grid_dep_wait();     // the selection is complete (this kernel may launch before it ends)
-  constexpr int SW = kMmaWarpStages;
   constexpr int R = NT * 8;
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_last;
-  __shared__ uint32_t meta_all[kMmaWarps][kMmaWarpStages];  // head mask | valid << 8 of each slot's tile
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  uint32_t* meta = meta_all[w];
-  const size_t bg = (size_t)b * p.Hkv + g;
+  constexpr int kOut = 2 + R;
   constexpr uint32_t k_bytes = kTile * D * 2;
   constexpr uint32_t c_bytes = kTile * R * 2;
   constexpr uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
-  constexpr uint32_t ring_bytes = kMmaWarps * SW * (stage_bytes + 8);
-  // shared memory: [rings | barriers] (page-mask scratch while the union is built) then the split's entries
-  uint32_t* ent = reinterpret_cast<uint32_t*>(smem + attn_ent_offset(ring_bytes, p.max_pages));
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ int s_last, s_fail;
+  __shared__ uint32_t meta_all[kMmaWarps][SW];  // head mask | valid tokens << 8 of each slot's tile
+  __shared__ int seg_all[kMmaWarps][SW];        // group of each slot's tile
   __shared__ int warp_tot[32];
-  __shared__ int s_cnt[8];
-  const UnionSlice sl = union_slice(p, b, g, G, split, reinterpret_cast<uint32_t*>(smem), ent, warp_tot, s_cnt);
-  const int U = sl.U, nsplit_active = sl.active;
-  if (sl.cnt == 0) {
-    if (split == 0 && U == 0)
-      for (int i = threadIdx.x; i < G * R; i += blockDim.x)
-        p.o_lat[((size_t)b * p.Hq + (size_t)g * G) * R + i] = 0.f;
-    return;
-  }
-  const int nent = sl.cnt;
-  const int ntiles = nent * p.tpp;
-
+  __shared__ int s_g0, s_p0, s_g1;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x, C = gridDim.x;
+  uint32_t* meta = meta_all[w];
+  int* segs = seg_all[w];
+  // shared memory: [rings | ring barriers | the CTA's result for the group being closed]
   unsigned char* ring = smem + (size_t)w * SW * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kMmaWarps * SW * stage_bytes) + w * SW;
+  float* part_s = reinterpret_cast<float*>(smem + (size_t)kMmaWarps * SW * (stage_bytes + 8));  // [G][kOut]
   if (lane == 0) {
     for (int s = 0; s < SW; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
   }
-  __syncwarp();
+  if (threadIdx.x == 0) {
+    s_fail = 0;
+    s_g0 = 0;
+    s_p0 = 0;
+    s_g1 = 0;
+  }
+  __syncthreads();
+  grid_dep_wait();     // the union lists are complete (this kernel may launch before their writer ends)
+  allow_dependents();  // the out-projection may launch and start streaming its weights
 
-  const int L = p.seq_len[b];
-  const int n = min((L + p.page - 1) / p.page, p.max_pages);
-  const int last_valid = L - (n - 1) * p.page;
+  // ---- the CTA's run of the global tile order --------------------------------
+  const int NG = p.ngroups;
+  auto tiles = [&](int g) { return (int)min(__ldcg(p.ucount + g), (uint32_t)p.umax) * p.tpp; };
+  int T, q, lo, hi;
+  {
+    const int per = (NG + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int r0 = min(NG, (int)threadIdx.x * per), r1 = min(NG, r0 + per);
+    int local = 0;
+    for (int g = r0; g < r1; ++g) local += tiles(g);
+    int P = block_exclusive_scan(local, warp_tot, T);
+    q = run_length(T, C);
+    lo = min(T, c * q);
+    hi = min(T, lo + q);
+    for (int g = r0; g < r1; ++g) {
+      const int t = tiles(g);
+      if (t == 0 && c == 0) {  // a group with nothing to attend to: its heads' outputs are zero
+        const int b = g / p.Hkv, gg = g - b * p.Hkv;
+        for (int i = 0; i < G * R; ++i) p.o_lat[((size_t)b * p.Hq + (size_t)gg * G) * R + i] = 0.f;
+      }
+      if (t > 0 && lo < hi) {
+        if (P <= lo && lo < P + t) {
+          s_g0 = g;
+          s_p0 = P;
+        }
+        if (P <= hi - 1 && hi - 1 < P + t) s_g1 = g;
+      }
+      P += t;
+    }
+  }
+  __syncthreads();
+  if (lo >= hi) return;  // nothing left for this CTA (uniform)
+  const int g_first = s_g0, g_last = s_g1;
+
   const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k_raw);
   const __nv_bfloat16* cbase = static_cast<const __nv_bfloat16*>(p.c_lat);
-
-  // this warp's tiles: t = w + kMmaWarps * i; lane j of a batch of 32 holds tile i = base + j
-  const int my_tiles = (ntiles > w) ? (ntiles - w + kMmaWarps - 1) / kMmaWarps : 0;
-  int d_phys = -1, d_valid = 0;
-  uint32_t d_mask = 0;
-  auto load_desc = [&](int base) {  // descriptors of tiles base .. base+31 of this warp
-    d_phys = -1;
-    d_valid = 0;
-    d_mask = 0;
-    const int i = base + lane;
-    if (i < my_tiles) {
-      const int t = w + kMmaWarps * i;
-      const int e = t / p.tpp, sub = t - e * p.tpp;
-      const uint32_t en = ent[e];
-      const int pg = (int)(en & 0xffffffu);
-      d_mask = en >> 24;
-      if (pg < n) {
-        const int ph = p.block_table[(size_t)b * p.max_pages + pg];
-        if (ph >= 0 && ph < p.num_phys) {
-          d_phys = ph * p.tpp + sub;  // tile index of the head-g page block, in 16-row units
-          d_valid = min(kTile, max(0, ((pg == n - 1) ? last_valid : p.page) - sub * kTile));
-        } else {
-          set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
-        }
-      }
-    }
-  };
   const uint64_t stream_pol = l2_evict_first();
-  // issue tile i of this warp into slot i % SW (lane 0); all lanes take part in the shuffles
+
+  // ---- descriptors of this warp's tiles, 32 at a time (lane j: the batch's tile j) ----
+  // The warp's tiles are t = lo + w + kMmaWarps * k.  A descriptor: the
+  // physical page (kNoPage: nothing to read), head mask | valid tokens << 8 |
+  // 16-row block of the page << 16, and the group.
+  const int my_tiles = (hi - lo > w) ? (hi - lo - w + kMmaWarps - 1) / kMmaWarps : 0;
+  int wg = g_first, wp = s_p0, wt = tiles(g_first);  // group of the previous batch's last tile
+  uint32_t d_id = kNoPage, d_meta = 0;
+  int d_grp = g_first;
+  auto load_desc = [&](int k0) {
+    const int k = k0 + lane;
+    int g = wg, P = wp, tt = wt;
+    d_id = kNoPage;
+    d_meta = 0;
+    if (k < my_tiles) {
+      const int t = lo + w + kMmaWarps * k;
+      while (t >= P + tt) {  // on to the group holding tile t (groups without tiles are stepped over)
+        P += tt;
+        ++g;
+        tt = tiles(g);
+      }
+      const uint32_t* list = p.lists + (size_t)g * p.ustride;
+      const int e = (t - P) / p.tpp, sub = (t - P) - e * p.tpp;
+      const uint32_t en = __ldcg(list + 4 + e);
+      const int pv = (e == tt / p.tpp - 1) ? (int)__ldcg(list + 1) : p.page;
+      const uint32_t id = en & kNoPage;
+      if (id != kNoPage && id >= (uint32_t)p.num_phys) set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
+      const int valid = (id < (uint32_t)p.num_phys) ? min(kTile, max(0, pv - sub * kTile)) : 0;
+      d_id = valid > 0 ? id : kNoPage;
+      d_meta = (en >> 24) | ((uint32_t)valid << 8) | ((uint32_t)sub << 16);
+    }
+    d_grp = g;
+    // the next batch walks on from the group of this batch's last tile
+    const int last = min(31, my_tiles - 1 - k0);
+    wg = __shfl_sync(kFull, g, last);
+    wp = __shfl_sync(kFull, P, last);
+    wt = __shfl_sync(kFull, tt, last);
+  };
+  // issue the warp's tile i into slot i % SW (lane 0 copies; all lanes shuffle)
   auto issue = [&](int i) {
     const int j = i & 31;
-    const int ph = __shfl_sync(kFull, d_phys, j);
-    const int valid = __shfl_sync(kFull, d_valid, j);
-    const uint32_t mask = __shfl_sync(kFull, d_mask, j);
+    const uint32_t id = __shfl_sync(kFull, d_id, j);
+    const uint32_t mt = __shfl_sync(kFull, d_meta, j);
+    const int grp = __shfl_sync(kFull, d_grp, j);
     if (lane == 0) {
-      meta[i % SW] = mask | ((uint32_t)valid << 8);
+      meta[i % SW] = (id == kNoPage) ? (mt & 0xffu) : (mt & 0xffffu);
+      segs[i % SW] = grp;
       uint64_t* bar = &full[i % SW];
       unsigned char* st = ring + (size_t)(i % SW) * stage_bytes;
       fence_proxy_async_smem();
-      if (valid > 0) {
-        const int pidx = ph / p.tpp, sub = ph - pidx * p.tpp;
-        const size_t row0 = ((size_t)pidx * p.Hkv + g) * p.page + (size_t)sub * kTile;
+      if (id != kNoPage) {
+        const int sub = (int)(mt >> 16);
+        const size_t row0 = ((size_t)id * p.Hkv + (size_t)(grp % p.Hkv)) * p.page + (size_t)sub * kTile;
         mbar_arrive_expect_tx(bar, k_bytes + c_bytes);
         bulk_g2s_hint(st, kbase + row0 * D, k_bytes, bar, stream_pol);  // read once: evict first
         bulk_g2s_hint(st + k_bytes, cbase + row0 * R, c_bytes, bar, stream_pol);
@@ -593,34 +682,110 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
     }
   };
 
+  // ---- the warp's running state for the current group (heads as fragment rows) ----
   const int gr = lane >> 2, tq = lane & 3;  // fragment row (head) and column pair
   const bool head_ok = gr < G;
+  float m_run = -INFINITY, l_run = 0.f;
+  float oacc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
   uint32_t qa[KS][2];
-  {
-    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G + gr) * D;
+  auto load_q = [&](int grp) {
+    const int b = grp / p.Hkv, gg = grp - b * p.Hkv;
+    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + (size_t)gg * G + gr) * D;
 #pragma unroll
     for (int s2 = 0; s2 < KS; ++s2) {
       qa[s2][0] = head_ok ? *reinterpret_cast<const uint32_t*>(qr + 16 * s2 + 2 * tq) : 0u;
       qa[s2][1] = head_ok ? *reinterpret_cast<const uint32_t*>(qr + 16 * s2 + 2 * tq + 8) : 0u;
     }
-  }
-  float m_run = -INFINITY, l_run = 0.f;
-  float oacc[NT][4];
+  };
+
+  // Closing a group (every warp of the CTA, the same groups in the same
+  // order): the warps' states are folded into part_s one warp after the other
+  // (a fixed order, so the result does not depend on timing), part_s goes to
+  // the CTA's partial slot of the group, and the last CTA of the group to get
+  // there merges the group's partials into o_lat.
+  int seg_g = g_first, seg_p = s_p0, seg_t = tiles(g_first);
+  auto close_group = [&]() {
+    l_run += __shfl_xor_sync(kFull, l_run, 1);
+    l_run += __shfl_xor_sync(kFull, l_run, 2);
+#pragma unroll 1
+    for (int ww = 0; ww < kMmaWarps; ++ww) {
+      if (w == ww) {
+        float* row = part_s + (size_t)gr * kOut;
+        float Mn = m_run, fs = 0.f, fw = 1.f;
+        if (head_ok) {
+          const float Ms = (ww == 0) ? -INFINITY : row[0];
+          Mn = fmaxf(Ms, m_run);
+          fs = (Ms == -INFINITY) ? 0.f : exp2f(Ms - Mn);
+          fw = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mn);
 #pragma unroll
-  for (int j = 0; j < NT; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+          for (int jj = 0; jj < NT; ++jj)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              float* a = row + 2 + 8 * jj + 2 * tq + e;
+              *a = (ww == 0 ? 0.f : *a * fs) + oacc[jj][e] * fw;
+            }
+        }
+        __syncwarp();  // the row's four lanes have read row[0] before it changes
+        if (head_ok && tq == 0) {
+          row[1] = (ww == 0 ? 0.f : row[1] * fs) + l_run * fw;
+          row[0] = Mn;
+        }
+      }
+      __syncthreads();
+    }
+    // slot c + group: unique, and the slots of a group's CTAs are consecutive
+    float* slot = p.part + ((size_t)(c + seg_g) * G) * kOut;
+    const bool failed = s_fail != 0;
+    for (int i = threadIdx.x; i < G * kOut; i += blockDim.x) {
+      float v = part_s[i];
+      if (failed && (i % kOut) == 1) v = __int_as_float(0x7fc00000);  // a wait gave up: the head's output is NaN
+      slot[i] = v;
+    }
+    const int ca = seg_p / q, cb = (seg_p + seg_t - 1) / q;  // the group's CTAs
+    const int b = seg_g / p.Hkv, gg = seg_g - b * p.Hkv;
+    if (last_of_group(p, (size_t)seg_g, cb - ca + 1, &s_last)) {
+      merge_group_splits(p, b, gg, G, R, ca + seg_g, cb - ca + 1, w, kMmaWarps, lane);
+      if (threadIdx.x == 0) p.cnt[seg_g] = 0;
+    }
+    __syncthreads();  // part_s is rewritten for the next group
+    m_run = -INFINITY;
+    l_run = 0.f;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
+    if (seg_g == g_last) {
+      seg_g = g_last + 1;  // the CTA's last group is closed
+      return;
+    }
+    // the next group with tiles (g_last has some, so the walk stops there at the latest)
+    do {
+      seg_p += seg_t;
+      ++seg_g;
+      seg_t = tiles(seg_g);
+    } while (seg_t == 0);
+    load_q(seg_g);
+  };
+
   constexpr int mk = 7;  // K rows have 8 or 16 chunks
   const int mc = swz_mask(R);
   const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix mi takes its row rr from this lane
   bool ok = true;
-
+  load_q(g_first);
+  int issued = 0, consumed = 0;
   if (my_tiles > 0) load_desc(0);
-  for (int i = 0; i < min(SW, my_tiles); ++i) issue(i);
-  for (int i = 0; i < my_tiles; ++i) {
-    const int s = i % SW;
-    if (!mbar_wait_bounded(&full[s], (uint32_t)((i / SW) & 1))) {
-      ok = false;
+  while (issued < SW && issued < my_tiles) {
+    issue(issued);
+    ++issued;
+  }
+  while (consumed < my_tiles) {
+    const int s = consumed % SW;
+    if (!__all_sync(kFull, mbar_wait_bounded(&full[s], (uint32_t)((consumed / SW) & 1)))) {
+      ok = false;  // the whole warp gives up together
       break;
     }
+    const int tgrp = segs[s];
+    while (seg_g < tgrp) close_group();  // groups of this CTA that the warp has no more tiles of
     const uint32_t mt = meta[s];
     const int valid = (int)(mt >> 8);
     if (valid > 0) {
@@ -694,72 +859,38 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) attn_mma_kernel(AttnParams 
         }
       }
     }
-    __syncwarp();  // every lane is done with slot s (and read meta[s])
-    // refill this slot with tile i + SW; a tile's descriptor is read from the lane
-    // registers only when it is issued, so reloading the next 32 here is safe
-    const int nx = i + SW;
-    if (nx < my_tiles) {
-      if ((nx & 31) == 0) load_desc(nx);
-      issue(nx);
+    __syncwarp();  // every lane is done with slot s (and has read meta[s], segs[s])
+    ++consumed;
+    // refill the slot just consumed (the next batch of descriptors replaces the
+    // lane registers only once every tile of this batch has been issued)
+    if (issued < my_tiles) {
+      if ((issued & 31) == 0) load_desc(issued);
+      issue(issued);
+      ++issued;
     }
   }
-  l_run += __shfl_xor_sync(kFull, l_run, 1);
-  l_run += __shfl_xor_sync(kFull, l_run, 2);
-  if (!ok) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
-
-  // merge the warps: each warp's (max, sum, acc[R]) per head -> one split result
-  constexpr int kOut = 2 + R;
-  float* mb = reinterpret_cast<float*>(smem);  // [kMmaWarps][G][kOut], reuses the rings
-  __syncthreads();
-  if (gr < G) {
-    float* dst = mb + ((size_t)w * G + gr) * kOut;
-    if (tq == 0) {
-      dst[0] = m_run;
-      dst[1] = l_run;
+  if (!ok) {
+    // a wait gave up: let this warp's copies still in flight land before its
+    // ring is released, and poison the results of the groups still open
+    if (lane == 0) {
+      s_fail = 1;
+      drain_ring(full, SW, consumed, issued);
     }
-#pragma unroll
-    for (int jj = 0; jj < NT; ++jj) {
-      dst[2 + 8 * jj + 2 * tq] = oacc[jj][0];
-      dst[3 + 8 * jj + 2 * tq] = oacc[jj][1];
-    }
+    __syncwarp();
   }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < G * R; idx += blockDim.x) {
-    const int hi = idx / R, dim = idx - hi * R;
-    float M = -INFINITY;
-#pragma unroll
-    for (int ww = 0; ww < kMmaWarps; ++ww) M = fmaxf(M, mb[((size_t)ww * G + hi) * kOut]);
-    float Ls = 0.f, As = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int ww = 0; ww < kMmaWarps; ++ww) {
-        const float* src = mb + ((size_t)ww * G + hi) * kOut;
-        const float f = exp2f(src[0] - M);  // 0 for a warp that saw nothing of this head
-        Ls += src[1] * f;
-        As += src[2 + dim] * f;
-      }
-    }
-    float* out = p.part + (((size_t)b * p.Hq + (size_t)g * G + hi) * p.nsplit + split) * (R + 2);
-    out[2 + dim] = As;
-    if (dim == 0) {
-      out[0] = M;
-      out[1] = Ls;
-    }
-  }
-  if (!last_of_group(p, bg, nsplit_active, &s_last)) return;
-  merge_group_splits(p, b, g, G, R, nsplit_active, w, kMmaWarps, lane);
-  if (threadIdx.x == 0) p.cnt[bg] = 0;
+  while (seg_g <= g_last) close_group();  // the same groups in every warp
+  if (!ok && lane == 0) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------
 // launch
 // ---------------------------------------------------------------------------
-// The attention kernels launch as programmatic dependents of the selection
-// kernel before them on the stream: their CTAs may start while it finishes and
-// wait (grid_dep_wait) before reading anything.
+// The attention kernels launch as programmatic dependents of the kernel that
+// writes the union lists: their CTAs may start while it finishes and wait
+// (grid_dep_wait) before reading them.
 template <typename K>
-static cudaError_t launch_dependent_of_route(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                                            const AttnParams& p) {
+static cudaError_t launch_dependent(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                    const AttnParams& p) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -773,69 +904,67 @@ static cudaError_t launch_dependent_of_route(K kernel, dim3 grid, dim3 block, si
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-size_t attn_smem_bytes(int d, int r, int esize, int max_pages, int eps) {
-  const size_t stage = ((size_t)kTile * (d + r) * esize + 127) & ~(size_t)127;
-  return attn_ent_offset((size_t)kStages * stage + 2 * kStages * 8, max_pages) + (size_t)eps * 4;
-}
-
 template <typename T, int D, int G, int CU>
-static cudaError_t launch_attn_t(const AttnParams& p, int batch, cudaStream_t st) {
-  const size_t smem = attn_smem_bytes(D, p.r, sizeof(T), p.max_pages, p.eps);
+static cudaError_t launch_attn_t(const AttnParams& p, int grid, cudaStream_t st) {
+  const size_t smem = core_smem_bytes(D, p.r, sizeof(T));
   cudaError_t e = ensure_smem((const void*)attn_kernel<T, D, G, CU>, smem);
   if (e != cudaSuccess) return e;
-  return launch_dependent_of_route(attn_kernel<T, D, G, CU>, dim3(p.nsplit, p.Hkv, batch), dim3(32 * (G + 1)),
-                                   smem, st, p);
+  return launch_dependent(attn_kernel<T, D, G, CU>, dim3(grid), dim3(32 * (G + 1)), smem, st, p);
 }
 
 template <typename T, int D, int G>
-static cudaError_t launch_attn_r(const AttnParams& p, int batch, cudaStream_t st) {
-  return (p.r <= 64) ? launch_attn_t<T, D, G, 1>(p, batch, st) : launch_attn_t<T, D, G, 2>(p, batch, st);
+static cudaError_t launch_attn_r(const AttnParams& p, int grid, cudaStream_t st) {
+  return (p.r <= 64) ? launch_attn_t<T, D, G, 1>(p, grid, st) : launch_attn_t<T, D, G, 2>(p, grid, st);
 }
 
 template <typename T, int D>
-static cudaError_t launch_attn_g(const AttnParams& p, int G, int batch, cudaStream_t st) {
+static cudaError_t launch_attn_g(const AttnParams& p, int G, int grid, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_attn_r<T, D, 1>(p, batch, st);
-    case 2: return launch_attn_r<T, D, 2>(p, batch, st);
-    case 4: return launch_attn_r<T, D, 4>(p, batch, st);
-    case 8: return launch_attn_r<T, D, 8>(p, batch, st);
+    case 1: return launch_attn_r<T, D, 1>(p, grid, st);
+    case 2: return launch_attn_r<T, D, 2>(p, grid, st);
+    case 4: return launch_attn_r<T, D, 4>(p, grid, st);
+    case 8: return launch_attn_r<T, D, 8>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D, int G, int NT>
-static cudaError_t launch_mma_t(const AttnParams& p, int batch, cudaStream_t st) {
-  const size_t stage = ((size_t)kTile * (D + NT * 8) * 2 + 127) & ~(size_t)127;
-  const size_t smem = attn_ent_offset((size_t)kMmaWarps * kMmaWarpStages * (stage + 8), p.max_pages) + (size_t)p.eps * 4;
+template <int D, int G, int NT, int SW>
+static cudaError_t launch_mma_t(const AttnParams& p, int grid, cudaStream_t st) {
+  const size_t smem = mma_smem_bytes(D, NT * 8, SW, G);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem((const void*)attn_mma_kernel<D, G, NT>, smem);
+  cudaError_t e = ensure_smem((const void*)attn_mma_kernel<D, G, NT, SW>, smem);
   if (e != cudaSuccess) return e;
-  return launch_dependent_of_route(attn_mma_kernel<D, G, NT>, dim3(p.nsplit, p.Hkv, batch), dim3(32 * kMmaWarps),
-                                   smem, st, p);
+  return launch_dependent(attn_mma_kernel<D, G, NT, SW>, dim3(grid), dim3(32 * kMmaWarps), smem,
+                          st, p);
+}
+
+template <int D, int G, int NT>
+static cudaError_t launch_mma_s(const AttnParams& p, int slots, int grid, cudaStream_t st) {
+  return (slots == 2) ? launch_mma_t<D, G, NT, 2>(p, grid, st) : launch_mma_t<D, G, NT, 3>(p, grid, st);
 }
 
 template <int D, int G>
-static cudaError_t launch_mma_r(const AttnParams& p, int batch, cudaStream_t st) {
+static cudaError_t launch_mma_r(const AttnParams& p, int slots, int grid, cudaStream_t st) {
   switch (p.r / 8) {
-    case 2: return launch_mma_t<D, G, 2>(p, batch, st);
-    case 4: return launch_mma_t<D, G, 4>(p, batch, st);
-    case 6: return launch_mma_t<D, G, 6>(p, batch, st);
-    case 8: return launch_mma_t<D, G, 8>(p, batch, st);
-    case 10: return launch_mma_t<D, G, 10>(p, batch, st);
-    case 12: return launch_mma_t<D, G, 12>(p, batch, st);
-    case 14: return launch_mma_t<D, G, 14>(p, batch, st);
-    case 16: return launch_mma_t<D, G, 16>(p, batch, st);
+    case 2: return launch_mma_s<D, G, 2>(p, slots, grid, st);
+    case 4: return launch_mma_s<D, G, 4>(p, slots, grid, st);
+    case 6: return launch_mma_s<D, G, 6>(p, slots, grid, st);
+    case 8: return launch_mma_s<D, G, 8>(p, slots, grid, st);
+    case 10: return launch_mma_s<D, G, 10>(p, slots, grid, st);
+    case 12: return launch_mma_s<D, G, 12>(p, slots, grid, st);
+    case 14: return launch_mma_s<D, G, 14>(p, slots, grid, st);
+    case 16: return launch_mma_s<D, G, 16>(p, slots, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int D>
-static cudaError_t launch_mma_g(const AttnParams& p, int G, int batch, cudaStream_t st) {
+static cudaError_t launch_mma_g(const AttnParams& p, int G, int slots, int grid, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_mma_r<D, 1>(p, batch, st);
-    case 2: return launch_mma_r<D, 2>(p, batch, st);
-    case 4: return launch_mma_r<D, 4>(p, batch, st);
-    case 8: return launch_mma_r<D, 8>(p, batch, st);
+    case 1: return launch_mma_r<D, 1>(p, slots, grid, st);
+    case 2: return launch_mma_r<D, 2>(p, slots, grid, st);
+    case 4: return launch_mma_r<D, 4>(p, slots, grid, st);
+    case 8: return launch_mma_r<D, 8>(p, slots, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -843,20 +972,20 @@ static cudaError_t launch_mma_g(const AttnParams& p, int G, int batch, cudaStrea
 cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* scratch, int batch,
                                cudaStream_t st) {
   char* base = static_cast<char*>(scratch);
-  int32_t* cnt = reinterpret_cast<int32_t*>(base + pl.cnt_off);
-  float* part = reinterpret_cast<float*>(base + pl.part_off);
-  AttnParams ap{a.q, a.k_raw, a.c_lat, a.block_table, a.seq_len, a.sel, a.sel_cnt, cnt, part, a.o_lat, a.err,
-                a.Hq, a.Hkv, a.page, a.r, a.max_pages, a.num_phys, a.top_k, pl.umax, pl.tpp, pl.eps, pl.nsplit,
-                pl.nsplit_lo, pl.rich_from, (float)(1.4426950408889634 / sqrt((double)a.d))};
-  cudaError_t e;
+  AttnParams ap{a.q, a.k_raw, a.c_lat, reinterpret_cast<const uint32_t*>(base + pl.list_off),
+                reinterpret_cast<const uint32_t*>(base + pl.ucount_off), reinterpret_cast<int32_t*>(base + pl.cnt_off),
+                reinterpret_cast<float*>(base + pl.part_off), a.o_lat,
+                a.err, a.Hq, a.Hkv, a.page, a.r, a.num_phys, pl.tpp, batch * a.Hkv, pl.extra, pl.ustride, pl.umax,
+                (float)(1.4426950408889634 / sqrt((double)a.d))};
   const int G = a.Hq / a.Hkv;
-  (void)e;
   if (kc_swizzled(a.bf16, a.d, a.r))
-    return (a.d == 128) ? launch_mma_g<128>(ap, G, batch, st) : launch_mma_g<64>(ap, G, batch, st);
+    return (a.d == 128) ? launch_mma_g<128>(ap, G, pl.ring_slots, pl.grid, st)
+                        : launch_mma_g<64>(ap, G, pl.ring_slots, pl.grid, st);
   if (a.bf16)
-    return (a.d == 128) ? launch_attn_g<__nv_bfloat16, 128>(ap, G, batch, st)
-                        : launch_attn_g<__nv_bfloat16, 64>(ap, G, batch, st);
-  return (a.d == 128) ? launch_attn_g<float, 128>(ap, G, batch, st) : launch_attn_g<float, 64>(ap, G, batch, st);
+    return (a.d == 128) ? launch_attn_g<__nv_bfloat16, 128>(ap, G, pl.grid, st)
+                        : launch_attn_g<__nv_bfloat16, 64>(ap, G, pl.grid, st);
+  return (a.d == 128) ? launch_attn_g<float, 128>(ap, G, pl.grid, st)
+                      : launch_attn_g<float, 64>(ap, G, pl.grid, st);
 }
 
 }  // namespace bkv

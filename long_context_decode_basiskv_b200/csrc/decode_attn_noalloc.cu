@@ -6,10 +6,11 @@
 // code that runs while a stream is being captured into a CUDA graph (where
 // cudaMalloc is not allowed), or a deployment with a fixed memory budget
 // that forbids allocation after start-up.  This entry point runs exactly the
-// kernels of basiskv_decode_attn, but its scratch (the union lists, their
-// counts and the per-split partial results) lives in one file-scope
-// __device__ array of fixed size that the library owns.  The caller still
-// passes the inputs and the output.
+// kernels of basiskv_decode_attn with a given selection (the union lists from
+// it, then the attention kernel), but their scratch (the union lists, the
+// per-group counters and tile cursors, the per-split partial results) lives in
+// one file-scope __device__ array of fixed size that the library owns.  The
+// caller still passes the inputs and the output.
 //
 // The array costs kNoAllocScratchBytes of memory on every GPU on which the
 // library is loaded, until the process exits.
@@ -31,7 +32,8 @@ void* g_addr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device.  In host code
 // the array's name only stands for the symbol; the address the kernels need
-// is looked up once per device, with that device current.
+// is looked up once per device, with that device current, in the context
+// current then (the device's primary context for CUDA runtime callers).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -56,19 +58,14 @@ using namespace bkv;
 extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
     const basiskv_config* cfg, const basiskv_cache* cache, const void* q, int32_t batch,
     const int32_t* sel, const int32_t* sel_cnt, float* o_lat, int32_t* err_flag, void* stream) {
-  if (!cfg || !cache) return BASISKV_ERR_INVALID_ARG;
-  if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->num_q_heads % cfg->num_kv_heads != 0 ||
-      cfg->rank_v <= 0 || cfg->page_size <= 0 || cfg->top_k <= 0 || batch < 0)
-    return BASISKV_ERR_INVALID_ARG;
-  if (batch == 0) return BASISKV_OK;
-  if (cache->max_pages <= 0) return BASISKV_ERR_INVALID_ARG;
+  // the checks of basiskv_decode_attn, in its order
+  basiskv_status s = check_decode_attn(cfg, cache, q, batch, sel, sel_cnt, o_lat, err_flag);
+  if (s != BASISKV_OK || batch == 0) return s;
+  // there is no routing workspace whose union lists this call could read
+  if (!sel) return BASISKV_ERR_INVALID_ARG;
 
   // the same scratch basiskv_decode_attn takes from its workspace
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const DecodePlan plan = decode_plan(cfg->num_q_heads, cfg->num_kv_heads, cfg->page_size, cfg->rank_v, cfg->top_k,
-                                      batch, cache->max_pages, cfg->dtype == BASISKV_BF16, cfg->head_dim,
-                                      sms > 0 ? sms : 148);
+  const DecodePlan plan = plan_decode_attn(cfg, batch, cache->max_pages);
   if (plan.bytes > kNoAllocScratchBytes) {
     fprintf(stderr,
             "basiskv_decode_attn_noalloc: this shape needs %zu bytes of scratch, more than the "
@@ -76,32 +73,12 @@ extern "C" BASISKV_API basiskv_status basiskv_decode_attn_noalloc(
             plan.bytes, kNoAllocScratchBytes);
     return BASISKV_ERR_WORKSPACE;
   }
-
-  // the remaining checks of basiskv_decode_attn: a supported shape (the
-  // workspace query returns 0 otherwise), pointers present and aligned
-  if (basiskv_workspace_bytes(cfg, batch, cache->max_pages) == 0) return BASISKV_ERR_UNSUPPORTED;
-  if (!q || !sel || !sel_cnt || !o_lat || !err_flag) return BASISKV_ERR_INVALID_ARG;
-  if (!cache->k_raw || !cache->c_lat || !cache->block_table || !cache->seq_len ||
-      cache->num_phys_pages <= 0)
-    return BASISKV_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(cache->k_raw) |
-       reinterpret_cast<uintptr_t>(cache->c_lat)) & 15u)
-    return BASISKV_ERR_INVALID_ARG;
-
   void* scratch = nullptr;
   cudaError_t e = scratch_address(&scratch);
   if (e != cudaSuccess) {
-    fprintf(stderr, "basiskv_decode_attn_noalloc: cudaGetSymbolAddress failed: %s\n",
-            cudaGetErrorString(e));
+    fprintf(stderr, "basiskv_decode_attn_noalloc: cudaGetSymbolAddress failed: %s\n", cudaGetErrorString(e));
     return BASISKV_ERR_CUDA;
   }
-  DecodeArgs a{q, cache->k_raw, cache->c_lat, cache->block_table, cache->seq_len, sel, sel_cnt, o_lat, err_flag,
-               cfg->num_q_heads, cfg->num_kv_heads, cfg->head_dim, cfg->page_size, cfg->rank_v,
-               cache->max_pages, cache->num_phys_pages, cfg->top_k, cfg->dtype == BASISKV_BF16};
-  e = launch_decode_attn(plan, a, scratch, batch, (cudaStream_t)stream);
-  if (e != cudaSuccess) {
-    fprintf(stderr, "basiskv_decode_attn_noalloc: CUDA error %s\n", cudaGetErrorString(e));
-    return BASISKV_ERR_CUDA;
-  }
-  return BASISKV_OK;
+  return run_decode_attn(plan, cfg, cache, q, batch, sel, sel_cnt, o_lat, static_cast<char*>(scratch), err_flag,
+                         stream);
 }

@@ -40,35 +40,57 @@ struct RouteParams {
   int all_pages;    // 0: skip the sink and recent pages (always kept; their scores are not needed)
   int group_mode;   // 0: one selection per query head; 1 / 2: one per KV group from the
                     // sum / maximum of its heads' scores, copied to every head of the group
+  // the union lists the selection kernel leaves for the attention kernel (union.cuh)
+  uint32_t* lists;  // [B][Hkv][ustride]
+  uint32_t* ucount; // [B][Hkv] entries of each list (compact)
+  int32_t* ucnt;    // [B][Hkv] per-group arrival counters, zero between calls
+  int32_t* acnt;    // [B][Hkv] the attention kernel's split counters, zeroed with the lists
+  int ustride;
 };
 cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st);
+
+// Union lists from a given selection (sel / sel_cnt rows of every head).
+struct UnionParams {
+  const int32_t* sel;
+  const int32_t* sel_cnt;
+  const int32_t* block_table;
+  const int32_t* seq_len;
+  uint32_t* lists;
+  uint32_t* ucount;  // [B][Hkv] entries of each list (compact)
+  int32_t* acnt;  // [B][Hkv] the attention kernel's split counters, zeroed here for the
+                  //   attention launch that reads the lists
+  int32_t* err;
+  int Hq, Hkv, page, max_pages, num_phys, top_k, ustride;
+};
+cudaError_t launch_union(const UnionParams& u, int batch, cudaStream_t st);
 
 struct AttnParams {
   const void* q;
   const void* k_raw;
   const void* c_lat;
-  const int32_t* block_table;
-  const int32_t* seq_len;
-  const int32_t* sel;
-  const int32_t* sel_cnt;
-  int32_t* cnt;  // [B][Hkv] finished-split counters, zero between calls
-  float* part;   // [B][Hq][nsplit][r + 2]
-  float* o_lat;  // [B][Hq][r]
+  const uint32_t* lists;   // [B][Hkv][ustride] union lists (union.cuh)
+  const uint32_t* ucount;  // [B][Hkv] entries of each list
+  int32_t* cnt;            // [B][Hkv] finished-split counters, zero between calls
+  float* part;             // [grid + B Hkv][G][r + 2] partial results (per CTA, or per CTA and group)
+  float* o_lat;            // [B][Hq][r]
   int32_t* err;
-  int Hq, Hkv, page, r, max_pages, num_phys, top_k, umax, tpp, eps, nsplit, nsplit_lo, rich_from;
+  int Hq, Hkv, page, r, num_phys, tpp, ngroups, extra, ustride, umax;
   float qscale;  // log2(e) / sqrt(d)
 };
 
-// Tiles per split and scratch layout of one decode_attn call; depends on the
-// shape only, so the workspace query and every launch agree on it.
+// Grid and scratch layout of one decode_attn call; depends on the shape only,
+// so the workspace query and every launch agree on it.  Tensor-core kernel:
+// one resident wave, each CTA an equal run of all groups' tiles.  CUDA-core
+// kernel: every group gets one CTA, and the `extra` remaining CTAs are shared
+// out at run time in proportion to the groups' tiles.
 struct DecodePlan {
-  int umax;    // max union pages per (sequence, KV head)
-  int tpp;     // 16-token tiles per page
-  int eps;        // union pages per split, at most
-  int nsplit;     // splits of the groups with the most (grid x extent; partial slots per head)
-  int nsplit_lo;  // splits of groups b * Hkv + g < rich_from (nsplit or nsplit - 1)
-  int rich_from;
-  size_t cnt_off, part_off, bytes;
+  int umax;       // max union pages per (sequence, KV head)
+  int tpp;        // 16-token tiles per page
+  int grid;       // CTAs of the attention launch
+  int extra;      // CUDA-core kernel: grid - groups
+  int ustride;    // words per union list
+  int ring_slots; // tensor-core kernel: bulk-copy slots per warp
+  size_t list_off, ucount_off, cnt_off, part_off, bytes;
 };
 DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, int max_pages, bool bf16, int d,
                        int num_sms);
@@ -77,17 +99,25 @@ struct DecodeArgs {
   const void* q;
   const void* k_raw;
   const void* c_lat;
-  const int32_t* block_table;
-  const int32_t* seq_len;
-  const int32_t* sel;
-  const int32_t* sel_cnt;
   float* o_lat;
   int32_t* err;
-  int Hq, Hkv, d, page, r, max_pages, num_phys, top_k;
+  int Hq, Hkv, d, page, r, num_phys;
   bool bf16;
 };
+// The attention kernel over the union lists already in the plan's scratch.
 cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* scratch, int batch,
                                cudaStream_t st);
+
+// Host helpers of the C ABI (api.cu) shared with the allocation-free entry point.
+int num_sms();
+basiskv_status cuda_status(cudaError_t e);
+basiskv_status check_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache, const void* q, int32_t batch,
+                                 const int32_t* sel, const int32_t* sel_cnt, const float* o_lat,
+                                 const int32_t* err_flag);
+DecodePlan plan_decode_attn(const basiskv_config* cfg, int32_t batch, int32_t max_pages);
+basiskv_status run_decode_attn(const DecodePlan& plan, const basiskv_config* cfg, const basiskv_cache* cache,
+                               const void* q, int32_t batch, const int32_t* sel, const int32_t* sel_cnt,
+                               float* o_lat, char* scratch, int32_t* err_flag, void* stream);
 
 struct OutProjParams {
   const float* o;

@@ -34,6 +34,7 @@
 // sel rows of all G heads, so the attention kernel reads k + 2 pages per
 // group.
 #include "kernels.cuh"
+#include "union.cuh"
 
 namespace bkv {
 
@@ -169,13 +170,6 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
 constexpr int kSelectThreads = 256;
 constexpr int kSelectWarps = kSelectThreads / 32;
 
-__device__ __forceinline__ uint32_t order_key(float v) {
-  if (v != v) return 0u;  // NaN: below every score
-  if (v == 0.f) v = 0.f;  // -0 ties with +0
-  const uint32_t u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
 // Sum of one int per thread over the block.  `red` is shared scratch of
 // 2 * kSelectWarps ints used alternately (`phase` flips it), so one barrier
 // per call suffices.
@@ -216,21 +210,44 @@ __device__ __forceinline__ void put_cnt(const RouteParams& p, const SelRows& r, 
   for (int c = 0; c < r.copies; ++c) p.sel_cnt[r.out + c] = v;
 }
 
-template <int KPT>
-__global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
-  __shared__ int red[2 * kSelectWarps];
-  __shared__ int warp_tot[32];
-  allow_dependents();  // the attention kernel may launch; it waits for this selection
-  const int b = blockIdx.y, tid = threadIdx.x;
-  const int L = p.seq_len[b];
-  const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
-  const int kk = p.top_k;
-  const SelRows rows = sel_rows(p, blockIdx.x, b);
-  if (n <= kk + 2) {
-    for (int i = tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, (i < n) ? i : -1);
-    if (tid == 0) put_cnt(p, rows, n);
-    return;
+// After its rows are written, a selection CTA counts itself on its KV group's
+// counter; the last of the group's G CTAs (the only one in the per-group
+// modes) builds the group's union list for the attention kernel and returns
+// the counter to zero.  All threads call this.
+__device__ __forceinline__ void select_union_tail(const RouteParams& p, int b, int x, uint32_t* masks,
+                                                  int32_t* bt_smem, int* warp_tot, int* s_flag) {
+  const int G = p.Hq / p.Hkv;
+  const int g = p.group_mode ? x : x / G;
+  const int need = p.group_mode ? 1 : G;
+  const size_t bg = (size_t)b * p.Hkv + g;
+  __syncthreads();  // orders this CTA's sel stores before thread 0's release
+  if (threadIdx.x == 0) {
+    int last = 1;
+    if (need > 1) {
+      __threadfence();
+      const int prev = atomicAdd(&p.ucnt[bg], 1);
+      if (prev >= need) set_err(p.err, BASISKV_DEVERR_WORKSPACE);
+      last = prev == need - 1;
+      if (last) {
+        p.ucnt[bg] = 0;
+        __threadfence();  // acquire: the other heads' rows are visible from here on
+      }
+    }
+    *s_flag = last;
   }
+  __syncthreads();
+  if (!*s_flag) return;
+  union_from_selection(p.sel, p.sel_cnt, p.block_table, p.seq_len[b], b, g, p.Hq, p.Hkv, p.page, p.max_pages,
+                       p.num_phys, p.top_k, p.lists + bg * p.ustride, p.ucount + bg, p.acnt, p.err, masks,
+                       bt_smem, warp_tot);
+}
+
+// The selection proper of route_select_kernel (n > top_k + 2 pages).
+template <int KPT>
+__device__ __forceinline__ void select_rows_reg(const RouteParams& p, const SelRows& rows, int b, int n, int* red,
+                                                int* warp_tot) {
+  const int tid = threadIdx.x;
+  const int kk = p.top_k;
   // thread t holds pages [t * KPT, t * KPT + KPT)
   const float* sc = p.scores + rows.in * p.max_pages;
   const int p0 = tid * KPT;
@@ -296,6 +313,28 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParam
   if (tid == 0) put_cnt(p, rows, total);
 }
 
+template <int KPT>
+__global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
+  __shared__ int red[2 * kSelectWarps];
+  __shared__ int warp_tot[32];
+  __shared__ uint32_t s_masks[kSelectThreads * KPT / 4];  // the union's page masks (tail)
+  __shared__ int32_t s_bt[kSelectThreads * KPT];           // the sequence's block-table row (tail)
+  __shared__ int s_flag;
+  allow_dependents();  // the union lists' reader may launch; it waits for this grid
+  const int b = blockIdx.y, tid = threadIdx.x;
+  const int L = p.seq_len[b];
+  const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
+  const int kk = p.top_k;
+  const SelRows rows = sel_rows(p, blockIdx.x, b);
+  if (n <= kk + 2) {
+    for (int i = tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, (i < n) ? i : -1);
+    if (tid == 0) put_cnt(p, rows, n);
+  } else {
+    select_rows_reg<KPT>(p, rows, b, n, red, warp_tot);
+  }
+  select_union_tail(p, b, blockIdx.x, s_masks, s_bt, warp_tot, &s_flag);
+}
+
 // ---------------------------------------------------------------------------
 // selection for block tables wider than the register-key kernel handles
 // ---------------------------------------------------------------------------
@@ -345,29 +384,18 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
 // exactly.  Finds T, the k-th largest score of pages 1..n-2, and how many pages
 // scoring exactly T are kept (the lowest indices), then writes the kept pages
 // plus 0 and n-1 in ascending order.
-__global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(RouteParams p) {
-  extern __shared__ __align__(16) float ssc[];  // [max_pages] scores of this head
-  __shared__ int hist[256];
-  __shared__ int warp_tot[32];
-  __shared__ float redf[64];
-  __shared__ float cand[kCandCap];
-  __shared__ int s_ncand, s_D, s_above, s_rem;
-  __shared__ float s_T;
-  allow_dependents();
-
-  const int b = blockIdx.y;
+// The selection proper of route_select_hist_kernel (n > top_k + 2 pages).
+__device__ __forceinline__ void select_rows_hist(const RouteParams& p, const SelRows& rows, int b, int n,
+                                                 const float* sc, float* ssc, int* hist, int* warp_tot, float* redf,
+                                                 float* cand, int* ps_ncand, int* ps_D, int* ps_above, int* ps_rem,
+                                                 float* ps_T) {
   const int tid = threadIdx.x;
-  const int L = p.seq_len[b];
-  const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
   const int kk = p.top_k;
-  const SelRows rows = sel_rows(p, blockIdx.x, b);
-  const float* sc = p.scores + rows.in * p.max_pages;
-
-  if (n <= kk + 2) {
-    for (int i = tid; i < kk + 2; i += blockDim.x) put_sel(p, rows, i, (i < n) ? i : -1);
-    if (tid == 0) put_cnt(p, rows, n);
-    return;
-  }
+  int& s_ncand = *ps_ncand;
+  int& s_D = *ps_D;
+  int& s_above = *ps_above;
+  int& s_rem = *ps_rem;
+  float& s_T = *ps_T;
   const int ncand = n - 2;  // pages 1 .. n-2 compete
 
   float mn = INFINITY, mx = -INFINITY;
@@ -526,6 +554,35 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(Route
   if (tid == 0) put_cnt(p, rows, tot);
 }
 
+
+__global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(RouteParams p) {
+  extern __shared__ __align__(16) float ssc[];  // [max_pages] scores of this head
+  __shared__ int hist[256];
+  __shared__ int warp_tot[32];
+  __shared__ float redf[64];
+  __shared__ float cand[kCandCap];
+  __shared__ int s_ncand, s_D, s_above, s_rem;
+  __shared__ float s_T;
+  __shared__ int s_flag;
+  allow_dependents();
+
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int L = p.seq_len[b];
+  const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
+  const int kk = p.top_k;
+  const SelRows rows = sel_rows(p, blockIdx.x, b);
+  const float* sc = p.scores + rows.in * p.max_pages;
+
+  if (n <= kk + 2) {
+    for (int i = tid; i < kk + 2; i += blockDim.x) put_sel(p, rows, i, (i < n) ? i : -1);
+    if (tid == 0) put_cnt(p, rows, n);
+  } else {
+    select_rows_hist(p, rows, b, n, sc, ssc, hist, warp_tot, redf, cand, &s_ncand, &s_D, &s_above, &s_rem, &s_T);
+  }
+  // the scores are no longer needed: their shared memory holds the union's page masks
+  select_union_tail(p, b, blockIdx.x, reinterpret_cast<uint32_t*>(ssc), nullptr, warp_tot, &s_flag);
+}
 
 // ---------------------------------------------------------------------------
 // launch

@@ -104,9 +104,11 @@ class DecodeEngine:
             bk.route_group(self.cfg, self.cache, self.q, _GROUP_REDUCE[self.routing], self.sel,
                            self.sel_cnt, self.ws, self.err, scores, stream)
 
-    def decode_attn(self, stream=None):
-        bk.decode_attn(self.cfg, self.cache, self.q, self.sel, self.sel_cnt, self.o_lat, self.ws,
-                       self.err, stream)
+    def decode_attn(self, stream=None, from_route: bool = True):
+        """Attention over the step's selection: by default the union lists route() left in
+        the workspace; from_route=False passes sel / sel_cnt (the library rebuilds them)."""
+        sel, cnt = (None, None) if from_route else (self.sel, self.sel_cnt)
+        bk.decode_attn(self.cfg, self.cache, self.q, sel, cnt, self.o_lat, self.ws, self.err, stream)
 
     def out_proj(self, stream=None):
         bk.out_proj(self.cfg, self.factors, self.o_lat, self.y, self.ws, stream)
@@ -151,6 +153,34 @@ class DecodeEngine:
                 self.step()
         self._graph.replay()
         return self.y
+
+    def graph_step_host(self, host_in: torch.Tensor, host_y: torch.Tensor):
+        """One decode step with host buffers, replayed from one CUDA graph: the copy of the
+        step's inputs from `host_in` (pinned, input_buffer()'s layout and dtype), the four
+        calls, and the copy of y into `host_y` (pinned, y's shape and dtype).  The graph is
+        captured on the first call for these two buffers; the caller refills host_in before
+        a call and reads host_y once the current stream is synchronised."""
+        if not (host_in.is_pinned() and host_y.is_pinned()):
+            raise ValueError("host buffers must be pinned")
+        if host_in.shape != self._inbuf.shape or host_in.dtype != self._inbuf.dtype:
+            raise ValueError("host_in must match input_buffer()")
+        if host_y.shape != self.y.shape or host_y.dtype != self.y.dtype:
+            raise ValueError("host_y must match y")
+        key = (host_in.data_ptr(), host_y.data_ptr())
+        if getattr(self, "_io_key", None) != key:
+            side = torch.cuda.Stream(device=self.device)
+            side.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(side):
+                self.step()  # first launches (shared-memory attributes) outside the capture
+            torch.cuda.current_stream(self.device).wait_stream(side)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                self._inbuf.copy_(host_in, non_blocking=True)
+                self.step()
+                host_y.copy_(self.y, non_blocking=True)
+            self._io_graph, self._io_key = g, key
+        self._io_graph.replay()
+        return host_y
 
     def kc_swizzled(self) -> bool:
         """bf16 K and C pages are stored with 16-byte chunks XOR-swizzled per row."""

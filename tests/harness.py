@@ -49,6 +49,27 @@ class OracleCase:
         return cache, out
 
 
+def oracle_on_selection(oc: OracleCase, b: int, cache, out, gpu_sel: np.ndarray, gpu_cnt: np.ndarray):
+    """The oracle's attention and out-projection of sequence b's decode step over the
+    GPU's page selection.  Where the two selections differ only by pages whose routing
+    scores tie within the near-tie rule, both are correct selections; the outputs the GPU
+    must then match are the oracle's on the pages the GPU chose.  Heads whose selection
+    is the oracle's keep the oracle's own results.  cache and out come from
+    oc.sequence(b) (the cache holds the step's new token).
+    Returns (o_lat [Hq, r], y [hidden])."""
+    wl = oc.wl
+    group = wl.num_q_heads // wl.num_kv_heads
+    q = to64(oc.case.q[b])
+    L = cache.length
+    o = np.array(out["o_lat"], dtype=np.float64, copy=True)
+    for h in range(wl.num_q_heads):
+        s = np.asarray(gpu_sel[h, :gpu_cnt[h]], dtype=np.int64)
+        if not np.array_equal(s, out["sel"][h]):
+            g = h // group
+            o[h] = O.sparse_attention(q[h], cache.K[g, :L], cache.C[g, :L], s, cache.page_size)[0]
+    return o, O.out_projection(o, oc.G)
+
+
 def selection_ok(gpu_sel: np.ndarray, gpu_cnt: int, want: np.ndarray, scores: np.ndarray,
                  rel: float = NEAR_TIE_REL):
     """(ok, exact): GPU selection vs oracle selection under the near-tie rule."""

@@ -1,15 +1,35 @@
-"""The C ABI library on the host (no GPU needed): it loads, exports every
-function include/basiskv.h declares, and its host-side validation rejects bad
-arguments before launching anything."""
+"""The C ABI library on the host: it loads, exports every function
+include/basiskv.h declares, and its host-side validation rejects bad arguments
+before launching anything.
+
+The calls below pass made-up device addresses, which only the entry points'
+own checks keep from reaching a kernel.  So these tests always run in a
+process that sees no GPU: in place when none is visible, otherwise in a child
+process started with CUDA_VISIBLE_DEVICES empty, where a check that let a call
+through would fail with a CUDA error instead of touching device memory."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
+import torch
 
 from long_context_decode_basiskv_b200 import binding as bk
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GPU_VISIBLE = os.environ.get("CUDA_VISIBLE_DEVICES") != "" and torch.cuda.is_available()
+
+
+def test_host_checks_in_a_process_without_gpu():
+    """With a GPU visible, run this file again in a child process that sees none."""
+    if not GPU_VISIBLE:
+        pytest.skip("no GPU visible: the checks run in this process")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", "-m", "not gpu",
+                        os.path.abspath(__file__)], env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 def _declared():
@@ -19,6 +39,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def L():
+    if GPU_VISIBLE:
+        pytest.skip("a GPU is visible: these calls run in test_host_checks_in_a_process_without_gpu")
     if not os.path.exists(bk.LIB_PATH):
         from long_context_decode_basiskv_b200 import build
         build.build()
@@ -26,6 +48,7 @@ def L():
 
 
 def test_header_declarations_match_binding():
+    # reads files only
     assert _declared() == sorted(bk.SYMBOLS)
 
 
@@ -35,7 +58,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.basiskv_abi_version() == 2
+    assert L.basiskv_abi_version() == 3
     assert L.basiskv_status_string(0) == b"ok"
     assert L.basiskv_status_string(4).startswith(b"workspace")
     assert L.basiskv_status_string(99) == b"unknown status"
@@ -192,3 +215,54 @@ def test_prefill_checks(L):
                              None) == bk.ERR_INVALID_ARG                       # no error flag
     assert L.basiskv_prefill(ctypes.byref(cfg), ctypes.byref(good), ctypes.byref(f), 256, 256, 1, 161, 256,
                              None) == bk.ERR_INVALID_ARG                       # more tokens than the block table holds
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(dtype=7), bk.ERR_INVALID_ARG),
+    (dict(head_dim=96), bk.ERR_UNSUPPORTED),
+    (dict(num_q_heads=30), bk.ERR_INVALID_ARG),
+])
+def test_noalloc_validates_like_decode_attn(L, bad, status):
+    """The allocation-free call refuses a bad configuration exactly as the workspace call does,
+    before it looks at the size of its scratch."""
+    cfg = _cfg(**bad)
+    cache = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    a = L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(cache), 256, 1, 256, 256, 256, 256, 1 << 30, 256, None)
+    b = L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(cache), 256, 1, 256, 256, 256, 256, None)
+    assert a == b == status
+
+
+def test_noalloc_and_decode_attn_share_cache_limits(L):
+    cfg = _cfg()
+    big = bk.CCache(256, 256, 256, 256, 256, 256, 10, 49153)          # more pages than routing supports
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(big), 256, 1, 256, 256, 256, 256, 1 << 40, 256,
+                                 None) == bk.ERR_UNSUPPORTED
+    assert L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(big), 256, 1, 256, 256, 256, 256,
+                                         None) == bk.ERR_UNSUPPORTED
+    many = bk.CCache(256, 256, 256, 256, 256, 256, 1 << 24, 10)       # page ids beyond 24 bits
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(many), 256, 1, 256, 256, 256, 256, 1 << 40, 256,
+                                 None) == bk.ERR_UNSUPPORTED
+    assert L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(many), 256, 1, 256, 256, 256, 256,
+                                         None) == bk.ERR_UNSUPPORTED
+    # no summary pointer: attention does not read summaries, so both calls accept it up to the workspace
+    nosum = bk.CCache(256, 256, 256, 0, 256, 256, 10, 10)
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(nosum), 256, 1, 256, 256, 256, None, 0, 256,
+                                 None) == bk.ERR_WORKSPACE
+
+
+def test_selection_pointers_come_in_pairs(L):
+    cfg = _cfg()
+    good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    # sel without sel_cnt (or the reverse) is refused by both calls
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(good), 256, 1, 256, None, 256, 256, 1 << 30, 256,
+                                 None) == bk.ERR_INVALID_ARG
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(good), 256, 1, None, 256, 256, 256, 1 << 30, 256,
+                                 None) == bk.ERR_INVALID_ARG
+    assert L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(good), 256, 1, 256, None, 256, 256,
+                                         None) == bk.ERR_INVALID_ARG
+    # the allocation-free call has no routing workspace to take a selection from
+    assert L.basiskv_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(good), 256, 1, None, None, 256, 256,
+                                         None) == bk.ERR_INVALID_ARG
+    # with both NULL the workspace call attends over the routing call's lists: workspace still required
+    assert L.basiskv_decode_attn(ctypes.byref(cfg), ctypes.byref(good), 256, 1, None, None, 256, None, 0, 256,
+                                 None) == bk.ERR_WORKSPACE

@@ -6,7 +6,8 @@ import numpy as np
 import pytest
 import torch
 
-from tests.harness import OracleCase, assert_close, assert_stored_equal, gt_plain, selection_ok, storage_of, to64
+from tests.harness import (OracleCase, assert_close, assert_stored_equal, gt_plain, oracle_on_selection,
+                           selection_ok, storage_of, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +39,7 @@ class Run:
         torch.cuda.synchronize()
         self.oc = OracleCase(self.case)
         self.ref = [self.oc.sequence(b) for b in range(wl.batch)]
+        self.outputs = (self.eng.sel.clone(), self.eng.sel_cnt.clone(), self.eng.o_lat.clone(), self.eng.y.clone())
 
 
 @pytest.fixture(scope="module", params=sorted(SMALL))
@@ -147,22 +149,27 @@ def O_y(G, o_lat):
 
 
 def test_end_to_end(run):
+    """Every sequence and head: the selection under the near-tie rule, then o_lat and y
+    against the oracle's attention and out-projection over the GPU's own selection (the
+    oracle's results themselves wherever the two selections are identical)."""
     eng, wl = run.eng, run.wl
-    sel = eng.sel.cpu().numpy()
-    cnt = eng.sel_cnt.cpu().numpy()
-    o_lat = eng.o_lat.cpu().numpy()
-    y = eng.y.cpu().numpy()
-    for b, (_, out) in enumerate(run.ref):
-        same = all(selection_ok(sel[b, h], cnt[b, h], out["sel"][h], out["scores"][h])[1]
-                   for h in range(wl.num_q_heads))
-        if same:
-            assert_close(o_lat[b], out["o_lat"], storage_of(wl), f"o_lat b={b}")
-            assert_close(y[b], out["y"], storage_of(wl), f"y b={b}")
+    sel, cnt, o_lat, y = (t.cpu().numpy() for t in run.outputs)
+    for b, (cache, out) in enumerate(run.ref):
+        for h in range(wl.num_q_heads):
+            assert selection_ok(sel[b, h], cnt[b, h], out["sel"][h], out["scores"][h])[0], f"b={b} h={h}"
+        o_want, y_want = oracle_on_selection(run.oc, b, cache, out, sel[b], cnt[b])
+        assert_close(o_lat[b], o_want, storage_of(wl), f"o_lat b={b}")
+        assert_close(y[b], y_want, storage_of(wl), f"y b={b}")
 
 
-def test_step_is_deterministic(run):
-    eng = run.eng
-    y0, s0, o0 = eng.y.clone(), eng.sel.clone(), eng.o_lat.clone()
+def test_step_repeats(run):
+    """A second step on the same inputs selects the same pages and gives the same outputs
+    to within the tolerance (the attention kernel splits a group's tiles among its warps at
+    run time, so the order of its floating-point sums may differ between calls)."""
+    eng, wl = run.eng, run.wl
+    s0, c0, o0, y0 = run.outputs
     eng.step()
     torch.cuda.synchronize()
-    assert torch.equal(eng.sel, s0) and torch.equal(eng.o_lat, o0) and torch.equal(eng.y, y0)
+    assert torch.equal(eng.sel, s0) and torch.equal(eng.sel_cnt, c0)
+    assert_close(eng.o_lat.cpu().numpy(), o0.cpu().numpy(), storage_of(wl), "o_lat, second step")
+    assert_close(eng.y.cpu().numpy(), y0.cpu().numpy(), storage_of(wl), "y, second step")

@@ -42,10 +42,23 @@ def test_noalloc_matches_workspace_call_twice(wl):
 
 
 def test_noalloc_refuses_shapes_beyond_its_scratch():
+    """A batch whose scratch would not fit the fixed array is refused before any launch.  Every
+    buffer is sized for that batch (empty sequences), so even a call that got through would only
+    touch valid memory."""
     wl = shrink(WORKLOADS["llama3_8b_32k"], batch=2, context=2000, top_k=16, name="noalloc_big")
     eng = DecodeEngine(make_case(wl, "cuda"))
     too_many = 4096                         # sequences whose partials need far more than 16 MiB
+    cfg = eng.cfg
+    q = torch.zeros((too_many, cfg.num_q_heads, cfg.head_dim), dtype=cfg.dtype, device="cuda")
+    sel = torch.full((too_many, cfg.num_q_heads, cfg.top_k + 2), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((too_many, cfg.num_q_heads), dtype=torch.int32, device="cuda")
+    o = torch.zeros((too_many, cfg.num_q_heads, cfg.rank_v), dtype=torch.float32, device="cuda")
+    bt = torch.zeros((too_many, eng.cache.max_pages), dtype=torch.int32, device="cuda")
+    sl = torch.zeros((too_many,), dtype=torch.int32, device="cuda")
+    c = eng.cache.c()
+    big = bk.CCache(c.k_raw, c.c_lat, c.r_res, c.summary, bt.data_ptr(), sl.data_ptr(), c.num_phys_pages,
+                    c.max_pages)
     st = bk.lib().basiskv_decode_attn_noalloc(
-        ctypes.byref(eng.cfg.c()), ctypes.byref(eng.cache.c()), eng.q.data_ptr(), too_many,
-        eng.sel.data_ptr(), eng.sel_cnt.data_ptr(), eng.o_lat.data_ptr(), eng.err.data_ptr(), None)
+        ctypes.byref(cfg.c()), ctypes.byref(big), q.data_ptr(), too_many, sel.data_ptr(), cnt.data_ptr(),
+        o.data_ptr(), eng.err.data_ptr(), None)
     assert st == bk.ERR_WORKSPACE
