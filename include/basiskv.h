@@ -253,9 +253,8 @@ BASISKV_API basiskv_status basiskv_route_group(const basiskv_config* cfg, const 
  * max_pages) stored there, without rebuilding it; giving only one of them is
  * BASISKV_ERR_INVALID_ARG.  workspace as for basiskv_route (the same buffer
  * may be passed to both).  err_flag may not be NULL.
- * A group's tiles are shared out among the kernel's warps at run time, so
- * o_lat may differ between calls in the last bits of fp32 (the order of the
- * softmax sums), never by more than the rounding of those sums.
+ * The split of the work depends only on the union sizes, so repeated calls
+ * on the same inputs give bitwise identical o_lat.
  */
 BASISKV_API basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,
                                    const void* q, int32_t batch, const int32_t* sel,

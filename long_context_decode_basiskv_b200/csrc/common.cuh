@@ -227,17 +227,14 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 }
 
 
-// Asynchronous 16-byte global -> shared copy (LDGSTS) with an L2 eviction
-// hint, tracked per thread with commit / wait groups.  Both addresses 16-byte
-// aligned.  The copy is skipped when `pred` is false.
-__device__ __forceinline__ void cp_async16_hint(void* dst, const void* src, uint64_t policy) {
-  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "l"(policy)
-               : "memory");
-}
-// 16-byte copy that reads L2 only (data written by other CTAs of the same launch)
+// Asynchronous 16-byte global -> shared copy (LDGSTS) that reads L2 only,
+// tracked per thread with commit / wait groups; both addresses 16-byte aligned.
 __device__ __forceinline__ void cp_async16_cg(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// the same for one 4-byte word (both addresses 4-byte aligned)
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -255,30 +252,29 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Named barrier `id` (1..15) over `nthreads` threads (whole warps, every lane
-// of each participating warp executes it).
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// The same barrier, returning whether `pred` was true in any participating thread.
-__device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool pred) {
+// Thread-block cluster helpers: this CTA's rank in its cluster; the cluster
+// barrier split into arrive (release) and wait (acquire), executed by every
+// thread of every CTA of the cluster; an OR into another CTA's shared memory
+// (the word at the address `local` has in this CTA, in CTA `rank`).
+__device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
-
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void red_or_cluster(uint32_t* local, uint32_t v, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("red.shared::cluster.or.b32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 
 // -------------------------------------------------------------------------

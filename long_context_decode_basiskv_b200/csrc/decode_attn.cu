@@ -11,23 +11,23 @@
 // every page chosen by any of the group's G query heads, once, with a head
 // mask and its physical id resolved.  The routing kernel writes the lists;
 // when the caller passes its own selection, union_kernel builds them from it.
-// One launch then streams the lists, the splits filling one resident wave
-// (decode_plan).  Each split's result per
-// head (max, sum, acc[r]) goes to scratch; the last CTA of a group to finish
-// (counted with an atomic) merges the group's splits with the log-sum-exp rule
-// and writes o_lat.  Two kernels:
-//   * attn_mma_kernel (bf16 with the swizzled K/C layout, the main path): the
-//     groups' 16-token tiles, laid end to end, are cut into equal contiguous
-//     runs, one per CTA, so every SM streams the same bytes whatever the
-//     union sizes (a CTA's run may cross group boundaries; it closes each
-//     group it leaves).  Four warps per CTA take the run's tiles round-robin,
-//     each with its own ring of bulk copies (cp.async.bulk, mbarrier
-//     completion, bounded waits, no multicast), and run all G heads of the
-//     group on the tensor cores (mma.sync m16n8k16).  The split of the work
-//     depends only on the union sizes, so the output is reproducible.
-//   * attn_kernel (fp32 and shapes without the swizzled layout): each split
-//     takes an equal share of the list; warp 0 produces into a shared ring,
-//     warps 1..G consume, one per query head, on the CUDA cores.
+// One launch then streams the lists in one resident wave of CTAs: every group
+// gets one CTA and the remaining CTAs are shared out in proportion to the
+// groups' tiles (assign_cta), so every split holds about the same number of
+// tiles; split s of a group takes an equal contiguous share of its list.
+// Each split's result per head (max, sum, acc[r]) goes to scratch; the last
+// CTA of a group to finish (counted with an atomic) merges the group's splits
+// with the log-sum-exp rule and writes o_lat.  Two kernels:
+//   * attn_mma_kernel (bf16 with the swizzled K/C layout, the main path): four
+//     warps per CTA take the share's 16-token tiles round-robin, each with its
+//     own ring of bulk copies (cp.async.bulk, mbarrier completion, bounded
+//     waits, no multicast), and run all G heads of the group on the tensor
+//     cores (mma.sync m16n8k16); the warps' states are folded in warp order.
+//     The split of the work depends only on the union sizes, so the output is
+//     reproducible.
+//   * attn_kernel (fp32 and shapes without the swizzled layout): warp 0
+//     produces the share's tiles into a shared ring, warps 1..G consume, one
+//     per query head, on the CUDA cores.
 // HBM-bound: every byte of the union's pages is read once.
 #include "kernels.cuh"
 #include "union.cuh"
@@ -39,17 +39,16 @@ constexpr int kStages = 4;          // ring depth per CTA of the CUDA-core kerne
 constexpr int kCoreCtasMax = 6;     // resident CTAs per SM of the CUDA-core attention kernel, at most
 constexpr int kMmaCtasPerSm = 3;    // ... and of the tensor-core one (registers)
 constexpr int kMmaWarps = 4;        // warps per CTA of the tensor-core kernel
-constexpr int kMinWarpTiles = 2;    // tiles per warp of the tensor-core kernel, at least
-constexpr int kMinSplitTiles = 8;   // tiles per split of the CUDA-core kernel (full unions), at least
+constexpr int kMinSplitTiles = 8;   // tiles per split (full unions), at least
 constexpr size_t kSmemPerSm = 228 * 1024;
 constexpr size_t kSmemPerCtaReserved = 1024;
 
 static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// shared memory of the tensor-core kernel: rings, their barriers, one group's result
+// shared memory of the tensor-core kernel: rings, their barriers, the chunk queue's barriers
 static size_t mma_smem_bytes(int d, int r, int slots, int G) {
   const size_t stage = ((size_t)kTile * (d + r) * 2 + 127) & ~(size_t)127;
-  return (size_t)kMmaWarps * slots * (stage + 8) + (size_t)G * (r + 2) * 4;
+  return (size_t)kMmaWarps * slots * (stage + 8) + (size_t)G * (r + 2) * 4;  // + the CTA's result
 }
 // ... and of the CUDA-core kernel: ring and full / empty barriers
 static size_t core_smem_bytes(int d, int r, int esize) {
@@ -60,10 +59,8 @@ static size_t core_smem_bytes(int d, int r, int esize) {
 // ---------------------------------------------------------------------------
 // plan: splits per (sequence, KV head) and the scratch layout
 // ---------------------------------------------------------------------------
-// Tensor-core kernel: the grid is one resident wave; each CTA takes an equal
-// run of the groups' tiles laid end to end and writes one partial result per
-// group its run touches, in slot CTA + group (so grid + groups slots).
-// CUDA-core kernel: one CTA per group at least, up to one resident wave; the
+// Both kernels: one CTA per group at least, up to one resident wave (more
+// waves when there are more than half as many groups as resident CTAs); the
 // CTAs past one per group are shared out among the groups in proportion to
 // their tiles when the kernel runs (assign_cta), each split keeping at least
 // kMinSplitTiles tiles of a full union.  Each CTA writes one partial result.
@@ -91,26 +88,25 @@ DecodePlan decode_plan(int Hq, int Hkv, int page, int r, int top_k, int batch, i
   if (per_sm < 1) per_sm = 1;
   const long long slots = (long long)num_sms * per_sm;
   const long long groups = (long long)batch * Hkv;
-  if (pl.ring_slots > 0) {
-    pl.grid = (int)slots;
-    pl.extra = 0;
-  } else {
-    long long per_group = ((long long)pl.umax * pl.tpp + kMinSplitTiles - 1) / kMinSplitTiles;
-    if (per_group < 1) per_group = 1;
-    long long grid = slots < groups * per_group ? slots : groups * per_group;
-    if (grid < groups) grid = groups;
-    pl.grid = (int)grid;
-    pl.extra = (int)(grid - groups);
-  }
+  long long per_group = ((long long)pl.umax * pl.tpp + kMinSplitTiles - 1) / kMinSplitTiles;
+  if (per_group < 1) per_group = 1;
+  // one resident wave, or more when there are many groups: with at least two
+  // CTAs per group on average the larger groups still get several, and the
+  // later waves start wherever an SM frees up
+  const long long waves = std::max(1LL, (2 * groups + slots - 1) / slots);
+  long long grid = std::min(waves * slots, groups * per_group);
+  if (grid < groups) grid = groups;
+  pl.grid = (int)grid;
+  pl.extra = (int)(grid - groups);
   size_t off = 0;
   pl.list_off = off;
   off += up256((size_t)batch * Hkv * pl.ustride * 4);
   pl.ucount_off = off;
   off += up256((size_t)batch * Hkv * 4);
-  pl.cnt_off = off;
+  pl.cnt_off = off;  // per group: finished splits
   off += up256((size_t)batch * Hkv * 4);
-  pl.part_off = off;
-  off += up256((size_t)(pl.grid + groups) * G * (r + 2) * 4);
+  pl.part_off = off;  // one partial result per CTA
+  off += up256((size_t)pl.grid * G * (r + 2) * 4);
   pl.bytes = off;
   return pl;
 }
@@ -162,7 +158,8 @@ __global__ void __launch_bounds__(kUnionThreads) union_kernel(UnionParams u) {
   const int g = blockIdx.x, b = blockIdx.y;
   union_from_selection(u.sel, u.sel_cnt, u.block_table, u.seq_len[b], b, g, u.Hq, u.Hkv, u.page, u.max_pages,
                        u.num_phys, u.top_k, u.lists + ((size_t)b * u.Hkv + g) * u.ustride,
-                       u.ucount + (size_t)b * u.Hkv + g, u.acnt, u.err, masks, nullptr, warp_tot);
+                       u.ucount + (size_t)b * u.Hkv + g, u.acnt, (size_t)gridDim.y * u.Hkv, u.err, masks,
+                       nullptr, warp_tot);
 }
 
 cudaError_t launch_union(const UnionParams& u, int batch, cudaStream_t st) {
@@ -535,19 +532,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Work of the tensor-core kernel: the groups' tiles laid end to end (b * Hkv
-// + g order, T in all) and cut into contiguous runs of q = ceil(T / C) tiles,
-// run c for CTA c.  Every CTA but the last ones streams the same number of
-// tiles however the union sizes of the groups differ (no split has more than
-// the least possible maximum), and the CTAs holding a group's tiles are
-// consecutive, each with at least one of them.
-// q is rounded up to whole rounds of the CTA's warps (the slowest warp sets the
-// CTA's time, so this costs nothing) and to kMinWarpTiles tiles per warp.
-__device__ __forceinline__ int run_length(int T, int C) {
-  const int per_warp = (T + kMmaWarps * C - 1) / (kMmaWarps * C);
-  return kMmaWarps * max(per_warp, kMinWarpTiles);
-}
-
+// Work of the tensor-core kernel: one resident wave of CTAs, each on one
+// group.  Every group gets one CTA and the remaining CTAs are shared out in
+// proportion to the groups' tiles (assign_cta, the same rule as the CUDA-core
+// kernel), so the splits of all groups hold about the same number of tiles;
+// split s of a group's ns takes an equal contiguous share of the group's
+// union list.  The four warps take the share's tiles round-robin, each with
+// its own ring of 1-D bulk copies (mbarrier completion, bounded waits, no
+// multicast), and run all G heads of the group on the tensor cores
+// (mma.sync m16n8k16).  At the end the warps' states are folded in warp order
+// into the CTA's partial result; the last CTA of the group merges the
+// group's partials into o_lat.  The split of the work depends only on the
+// union sizes, so the output is reproducible.
 template <int D, int G, int NT, int SW>
 __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel(AttnParams p) {
   constexpr int KS = D / 16;
@@ -557,16 +553,13 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
   constexpr uint32_t c_bytes = kTile * R * 2;
   constexpr uint32_t stage_bytes = (k_bytes + c_bytes + 127u) & ~127u;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ int s_last, s_fail;
   __shared__ uint32_t meta_all[kMmaWarps][SW];  // head mask | valid tokens << 8 of each slot's tile
-  __shared__ int seg_all[kMmaWarps][SW];        // group of each slot's tile
   __shared__ int warp_tot[32];
-  __shared__ int s_g0, s_p0, s_g1;
+  __shared__ int s_asg[4];
+  __shared__ int s_last, s_fail;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int c = blockIdx.x, C = gridDim.x;
   uint32_t* meta = meta_all[w];
-  int* segs = seg_all[w];
-  // shared memory: [rings | ring barriers | the CTA's result for the group being closed]
+  // shared memory: [rings | ring barriers | the CTA's result]
   unsigned char* ring = smem + (size_t)w * SW * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kMmaWarps * SW * stage_bytes) + w * SW;
   float* part_s = reinterpret_cast<float*>(smem + (size_t)kMmaWarps * SW * (stage_bytes + 8));  // [G][kOut]
@@ -574,105 +567,57 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
     for (int s = 0; s < SW; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
   }
-  if (threadIdx.x == 0) {
-    s_fail = 0;
-    s_g0 = 0;
-    s_p0 = 0;
-    s_g1 = 0;
-  }
+  if (threadIdx.x == 0) s_fail = 0;
   __syncthreads();
   grid_dep_wait();     // the union lists are complete (this kernel may launch before their writer ends)
   allow_dependents();  // the out-projection may launch and start streaming its weights
-
-  // ---- the CTA's run of the global tile order --------------------------------
-  const int NG = p.ngroups;
-  auto tiles = [&](int g) { return (int)min(__ldcg(p.ucount + g), (uint32_t)p.umax) * p.tpp; };
-  int T, q, lo, hi;
-  {
-    const int per = (NG + (int)blockDim.x - 1) / (int)blockDim.x;
-    const int r0 = min(NG, (int)threadIdx.x * per), r1 = min(NG, r0 + per);
-    int local = 0;
-    for (int g = r0; g < r1; ++g) local += tiles(g);
-    int P = block_exclusive_scan(local, warp_tot, T);
-    q = run_length(T, C);
-    lo = min(T, c * q);
-    hi = min(T, lo + q);
-    for (int g = r0; g < r1; ++g) {
-      const int t = tiles(g);
-      if (t == 0 && c == 0) {  // a group with nothing to attend to: its heads' outputs are zero
-        const int b = g / p.Hkv, gg = g - b * p.Hkv;
-        for (int i = 0; i < G * R; ++i) p.o_lat[((size_t)b * p.Hq + (size_t)gg * G) * R + i] = 0.f;
-      }
-      if (t > 0 && lo < hi) {
-        if (P <= lo && lo < P + t) {
-          s_g0 = g;
-          s_p0 = P;
-        }
-        if (P <= hi - 1 && hi - 1 < P + t) s_g1 = g;
-      }
-      P += t;
-    }
-  }
-  __syncthreads();
-  if (lo >= hi) return;  // nothing left for this CTA (uniform)
-  const int g_first = s_g0, g_last = s_g1;
+  assign_cta(p, blockIdx.x, warp_tot, s_asg);
+  const int bg = s_asg[0], split = s_asg[1], ns = s_asg[2], slot0 = s_asg[3];
+  const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+  const uint32_t* list = p.lists + (size_t)bg * p.ustride;
+  const int U = min((int)__ldcg(list), p.umax);
+  const int tail_valid = (int)__ldcg(list + 1);
+  const int T = U * p.tpp;
+  const int per = (T + ns - 1) / ns;
+  const int lo = min(T, split * per), hi = min(T, lo + per);
+  const int my_tiles = (hi - lo > w) ? (hi - lo - w + kMmaWarps - 1) / kMmaWarps : 0;  // tiles lo + w + 4k
 
   const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k_raw);
   const __nv_bfloat16* cbase = static_cast<const __nv_bfloat16*>(p.c_lat);
   const uint64_t stream_pol = l2_evict_first();
 
-  // ---- descriptors of this warp's tiles, 32 at a time (lane j: the batch's tile j) ----
-  // The warp's tiles are t = lo + w + kMmaWarps * k.  A descriptor: the
-  // physical page (kNoPage: nothing to read), head mask | valid tokens << 8 |
-  // 16-row block of the page << 16, and the group.
-  const int my_tiles = (hi - lo > w) ? (hi - lo - w + kMmaWarps - 1) / kMmaWarps : 0;
-  int wg = g_first, wp = s_p0, wt = tiles(g_first);  // group of the previous batch's last tile
+  // descriptors of this warp's tiles, 32 at a time (lane j: the batch's tile j):
+  // the physical page (kNoPage: nothing to read), head mask | valid tokens << 8 | 16-row block << 16
   uint32_t d_id = kNoPage, d_meta = 0;
-  int d_grp = g_first;
   auto load_desc = [&](int k0) {
     const int k = k0 + lane;
-    int g = wg, P = wp, tt = wt;
     d_id = kNoPage;
     d_meta = 0;
     if (k < my_tiles) {
       const int t = lo + w + kMmaWarps * k;
-      while (t >= P + tt) {  // on to the group holding tile t (groups without tiles are stepped over)
-        P += tt;
-        ++g;
-        tt = tiles(g);
-      }
-      const uint32_t* list = p.lists + (size_t)g * p.ustride;
-      const int e = (t - P) / p.tpp, sub = (t - P) - e * p.tpp;
+      const int e = t / p.tpp, sub = t - e * p.tpp;
       const uint32_t en = __ldcg(list + 4 + e);
-      const int pv = (e == tt / p.tpp - 1) ? (int)__ldcg(list + 1) : p.page;
+      const int pv = (e == U - 1) ? tail_valid : p.page;
       const uint32_t id = en & kNoPage;
       if (id != kNoPage && id >= (uint32_t)p.num_phys) set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
       const int valid = (id < (uint32_t)p.num_phys) ? min(kTile, max(0, pv - sub * kTile)) : 0;
       d_id = valid > 0 ? id : kNoPage;
       d_meta = (en >> 24) | ((uint32_t)valid << 8) | ((uint32_t)sub << 16);
     }
-    d_grp = g;
-    // the next batch walks on from the group of this batch's last tile
-    const int last = min(31, my_tiles - 1 - k0);
-    wg = __shfl_sync(kFull, g, last);
-    wp = __shfl_sync(kFull, P, last);
-    wt = __shfl_sync(kFull, tt, last);
   };
   // issue the warp's tile i into slot i % SW (lane 0 copies; all lanes shuffle)
   auto issue = [&](int i) {
     const int j = i & 31;
     const uint32_t id = __shfl_sync(kFull, d_id, j);
     const uint32_t mt = __shfl_sync(kFull, d_meta, j);
-    const int grp = __shfl_sync(kFull, d_grp, j);
     if (lane == 0) {
       meta[i % SW] = (id == kNoPage) ? (mt & 0xffu) : (mt & 0xffffu);
-      segs[i % SW] = grp;
       uint64_t* bar = &full[i % SW];
       unsigned char* st = ring + (size_t)(i % SW) * stage_bytes;
       fence_proxy_async_smem();
       if (id != kNoPage) {
         const int sub = (int)(mt >> 16);
-        const size_t row0 = ((size_t)id * p.Hkv + (size_t)(grp % p.Hkv)) * p.page + (size_t)sub * kTile;
+        const size_t row0 = ((size_t)id * p.Hkv + (size_t)g) * p.page + (size_t)sub * kTile;
         mbar_arrive_expect_tx(bar, k_bytes + c_bytes);
         bulk_g2s_hint(st, kbase + row0 * D, k_bytes, bar, stream_pol);  // read once: evict first
         bulk_g2s_hint(st + k_bytes, cbase + row0 * R, c_bytes, bar, stream_pol);
@@ -682,7 +627,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
     }
   };
 
-  // ---- the warp's running state for the current group (heads as fragment rows) ----
+  // the warp's running state (heads as fragment rows) and the group's query
   const int gr = lane >> 2, tq = lane & 3;  // fragment row (head) and column pair
   const bool head_ok = gr < G;
   float m_run = -INFINITY, l_run = 0.f;
@@ -690,88 +635,19 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
 #pragma unroll
   for (int j = 0; j < NT; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
   uint32_t qa[KS][2];
-  auto load_q = [&](int grp) {
-    const int b = grp / p.Hkv, gg = grp - b * p.Hkv;
-    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + (size_t)gg * G + gr) * D;
+  {
+    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G + gr) * D;
 #pragma unroll
     for (int s2 = 0; s2 < KS; ++s2) {
       qa[s2][0] = head_ok ? *reinterpret_cast<const uint32_t*>(qr + 16 * s2 + 2 * tq) : 0u;
       qa[s2][1] = head_ok ? *reinterpret_cast<const uint32_t*>(qr + 16 * s2 + 2 * tq + 8) : 0u;
     }
-  };
-
-  // Closing a group (every warp of the CTA, the same groups in the same
-  // order): the warps' states are folded into part_s one warp after the other
-  // (a fixed order, so the result does not depend on timing), part_s goes to
-  // the CTA's partial slot of the group, and the last CTA of the group to get
-  // there merges the group's partials into o_lat.
-  int seg_g = g_first, seg_p = s_p0, seg_t = tiles(g_first);
-  auto close_group = [&]() {
-    l_run += __shfl_xor_sync(kFull, l_run, 1);
-    l_run += __shfl_xor_sync(kFull, l_run, 2);
-#pragma unroll 1
-    for (int ww = 0; ww < kMmaWarps; ++ww) {
-      if (w == ww) {
-        float* row = part_s + (size_t)gr * kOut;
-        float Mn = m_run, fs = 0.f, fw = 1.f;
-        if (head_ok) {
-          const float Ms = (ww == 0) ? -INFINITY : row[0];
-          Mn = fmaxf(Ms, m_run);
-          fs = (Ms == -INFINITY) ? 0.f : exp2f(Ms - Mn);
-          fw = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mn);
-#pragma unroll
-          for (int jj = 0; jj < NT; ++jj)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              float* a = row + 2 + 8 * jj + 2 * tq + e;
-              *a = (ww == 0 ? 0.f : *a * fs) + oacc[jj][e] * fw;
-            }
-        }
-        __syncwarp();  // the row's four lanes have read row[0] before it changes
-        if (head_ok && tq == 0) {
-          row[1] = (ww == 0 ? 0.f : row[1] * fs) + l_run * fw;
-          row[0] = Mn;
-        }
-      }
-      __syncthreads();
-    }
-    // slot c + group: unique, and the slots of a group's CTAs are consecutive
-    float* slot = p.part + ((size_t)(c + seg_g) * G) * kOut;
-    const bool failed = s_fail != 0;
-    for (int i = threadIdx.x; i < G * kOut; i += blockDim.x) {
-      float v = part_s[i];
-      if (failed && (i % kOut) == 1) v = __int_as_float(0x7fc00000);  // a wait gave up: the head's output is NaN
-      slot[i] = v;
-    }
-    const int ca = seg_p / q, cb = (seg_p + seg_t - 1) / q;  // the group's CTAs
-    const int b = seg_g / p.Hkv, gg = seg_g - b * p.Hkv;
-    if (last_of_group(p, (size_t)seg_g, cb - ca + 1, &s_last)) {
-      merge_group_splits(p, b, gg, G, R, ca + seg_g, cb - ca + 1, w, kMmaWarps, lane);
-      if (threadIdx.x == 0) p.cnt[seg_g] = 0;
-    }
-    __syncthreads();  // part_s is rewritten for the next group
-    m_run = -INFINITY;
-    l_run = 0.f;
-#pragma unroll
-    for (int j = 0; j < NT; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
-    if (seg_g == g_last) {
-      seg_g = g_last + 1;  // the CTA's last group is closed
-      return;
-    }
-    // the next group with tiles (g_last has some, so the walk stops there at the latest)
-    do {
-      seg_p += seg_t;
-      ++seg_g;
-      seg_t = tiles(seg_g);
-    } while (seg_t == 0);
-    load_q(seg_g);
-  };
+  }
 
   constexpr int mk = 7;  // K rows have 8 or 16 chunks
   const int mc = swz_mask(R);
   const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix mi takes its row rr from this lane
   bool ok = true;
-  load_q(g_first);
   int issued = 0, consumed = 0;
   if (my_tiles > 0) load_desc(0);
   while (issued < SW && issued < my_tiles) {
@@ -784,8 +660,6 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
       ok = false;  // the whole warp gives up together
       break;
     }
-    const int tgrp = segs[s];
-    while (seg_g < tgrp) close_group();  // groups of this CTA that the warp has no more tiles of
     const uint32_t mt = meta[s];
     const int valid = (int)(mt >> 8);
     if (valid > 0) {
@@ -859,7 +733,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
         }
       }
     }
-    __syncwarp();  // every lane is done with slot s (and has read meta[s], segs[s])
+    __syncwarp();  // every lane is done with slot s (and has read meta[s])
     ++consumed;
     // refill the slot just consumed (the next batch of descriptors replaces the
     // lane registers only once every tile of this batch has been issued)
@@ -871,15 +745,56 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
   }
   if (!ok) {
     // a wait gave up: let this warp's copies still in flight land before its
-    // ring is released, and poison the results of the groups still open
+    // ring is released, and mark the CTA's result
     if (lane == 0) {
       s_fail = 1;
+      set_err(p.err, BASISKV_DEVERR_TIMEOUT);
       drain_ring(full, SW, consumed, issued);
     }
     __syncwarp();
   }
-  while (seg_g <= g_last) close_group();  // the same groups in every warp
-  if (!ok && lane == 0) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
+  // the warps' states folded into part_s one warp after the other (a fixed
+  // order, so the result does not depend on timing)
+  l_run += __shfl_xor_sync(kFull, l_run, 1);
+  l_run += __shfl_xor_sync(kFull, l_run, 2);
+  __syncthreads();
+#pragma unroll 1
+  for (int ww = 0; ww < kMmaWarps; ++ww) {
+    if (w == ww) {
+      float* row = part_s + (size_t)gr * kOut;
+      float Mn = m_run, fs = 0.f, fw = 1.f;
+      if (head_ok) {
+        const float Ms = (ww == 0) ? -INFINITY : row[0];
+        Mn = fmaxf(Ms, m_run);
+        fs = (Ms == -INFINITY) ? 0.f : exp2f(Ms - Mn);
+        fw = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mn);
+#pragma unroll
+        for (int jj = 0; jj < NT; ++jj)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float* a = row + 2 + 8 * jj + 2 * tq + e;
+            *a = (ww == 0 ? 0.f : *a * fs) + oacc[jj][e] * fw;
+          }
+      }
+      __syncwarp();  // the row's four lanes have read row[0] before it changes
+      if (head_ok && tq == 0) {
+        row[1] = (ww == 0 ? 0.f : row[1] * fs) + l_run * fw;
+        row[0] = Mn;
+      }
+    }
+    __syncthreads();
+  }
+  float* slot = p.part + (size_t)blockIdx.x * G * kOut;  // the group's CTAs, and slots, are consecutive
+  const bool failed = s_fail != 0;
+  for (int i = threadIdx.x; i < G * kOut; i += blockDim.x) {
+    float v = part_s[i];
+    if (failed && (i % kOut) == 1) v = __int_as_float(0x7fc00000);  // a wait gave up: the head's output is NaN
+    slot[i] = v;
+  }
+  // the last CTA of the group to finish merges every split of its G heads
+  if (!last_of_group(p, (size_t)bg, ns, &s_last)) return;
+  merge_group_splits(p, b, g, G, R, slot0, ns, w, kMmaWarps, lane);
+  if (threadIdx.x == 0) p.cnt[bg] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -974,8 +889,8 @@ cudaError_t launch_decode_attn(const DecodePlan& pl, const DecodeArgs& a, void* 
   char* base = static_cast<char*>(scratch);
   AttnParams ap{a.q, a.k_raw, a.c_lat, reinterpret_cast<const uint32_t*>(base + pl.list_off),
                 reinterpret_cast<const uint32_t*>(base + pl.ucount_off), reinterpret_cast<int32_t*>(base + pl.cnt_off),
-                reinterpret_cast<float*>(base + pl.part_off), a.o_lat,
-                a.err, a.Hq, a.Hkv, a.page, a.r, a.num_phys, pl.tpp, batch * a.Hkv, pl.extra, pl.ustride, pl.umax,
+                reinterpret_cast<float*>(base + pl.part_off), a.o_lat, a.err, a.Hq, a.Hkv, a.page, a.r,
+                a.num_phys, pl.tpp, batch * a.Hkv, pl.extra, pl.ustride, pl.umax,
                 (float)(1.4426950408889634 / sqrt((double)a.d))};
   const int G = a.Hq / a.Hkv;
   if (kc_swizzled(a.bf16, a.d, a.r))

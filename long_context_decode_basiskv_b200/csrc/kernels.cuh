@@ -70,8 +70,8 @@ struct AttnParams {
   const void* c_lat;
   const uint32_t* lists;   // [B][Hkv][ustride] union lists (union.cuh)
   const uint32_t* ucount;  // [B][Hkv] entries of each list
-  int32_t* cnt;            // [B][Hkv] finished-split counters, zero between calls
-  float* part;             // [grid + B Hkv][G][r + 2] partial results (per CTA, or per CTA and group)
+  int32_t* cnt;            // [B Hkv] finished-split counters, zeroed when the lists are written
+  float* part;             // [grid][G][r + 2] partial results, one per CTA
   float* o_lat;            // [B][Hq][r]
   int32_t* err;
   int Hq, Hkv, page, r, num_phys, tpp, ngroups, extra, ustride, umax;
@@ -79,10 +79,10 @@ struct AttnParams {
 };
 
 // Grid and scratch layout of one decode_attn call; depends on the shape only,
-// so the workspace query and every launch agree on it.  Tensor-core kernel:
-// one resident wave, each CTA an equal run of all groups' tiles.  CUDA-core
-// kernel: every group gets one CTA, and the `extra` remaining CTAs are shared
-// out at run time in proportion to the groups' tiles.
+// so the workspace query and every launch agree on it.  Both attention
+// kernels: every group gets one CTA, and the `extra` remaining CTAs of one
+// resident wave are shared out at run time in proportion to the groups'
+// tiles; one partial result per CTA.
 struct DecodePlan {
   int umax;       // max union pages per (sequence, KV head)
   int tpp;        // 16-token tiles per page

@@ -28,8 +28,8 @@
 //
 // The page summaries S = mean(C) P_g + mean(R) E_g^T over each touched page's
 // valid tokens (old and new) are recomputed afterwards by a second kernel, in
-// fp64 from the stored C and R, one CTA per (sequence, KV head, 32 pages) with
-// the factors staged once.
+// fp64 from the stored C and R, one CTA per (sequence, KV head, 128 tokens of
+// pages) with the pages' blocks and the factors staged once.
 #include "kernels.cuh"
 #include "tcgen05.cuh"
 
@@ -348,10 +348,23 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
 // ---------------------------------------------------------------------------
 // page summaries of every page the appended tokens touched
 // ---------------------------------------------------------------------------
-constexpr int kSumPages = 32;  // pages per CTA
+// One CTA per (sequence, KV head, run of kSumTokens / page pages).  All of the
+// run's stored C and R blocks (contiguous per page) come into shared memory in
+// one round of 16-byte cp.async copies, then: the column means of each page's
+// valid tokens in fp64 (tokens in order), and S[x] = sum_j mean(C)_j P[j][x] +
+// sum_q mean(R)_q E[x][q] in fp64, rounded once.  E is staged transposed so
+// that consecutive x read consecutive words.
+constexpr int kSumTokens = 128;  // tokens (pages x page size) per CTA
 constexpr int kSumThreads = 128;
 
-__global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams p) {
+static int sum_pages(int page) { return std::max(1, kSumTokens / page); }
+static size_t sum_smem_bytes(int d, int r, int s, int page) {
+  const int np = sum_pages(page);
+  return (size_t)(r * d + d * s) * sizeof(float) + (size_t)np * page * (r + s) * 2 +
+         (size_t)np * (r + s) * sizeof(double) + 16 * sizeof(int);
+}
+
+__global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams p, int np) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int b = blockIdx.z, g = blockIdx.y, tid = threadIdx.x;
   const int d = p.d, r = p.r, s = p.s, P = p.page;
@@ -359,42 +372,74 @@ __global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams 
   if (L < p.n_new || L > p.max_pages * P || p.n_new <= 0) return;  // reported by the latent kernel
   const int first_page = (L - p.n_new) / P;
   const int last_page = (L - 1) / P;
-  const int pg0 = first_page + blockIdx.x * kSumPages;
+  const int pg0 = first_page + blockIdx.x * np;
   if (pg0 > last_page) return;
-  float* sP = reinterpret_cast<float*>(smem);  // [r][d]
-  float* sE = sP + r * d;                      // [d][s]
-  double* sMean = reinterpret_cast<double*>(sE + d * s);  // [r + s]
+  const int npg = min(np, last_page - pg0 + 1);  // pages of this CTA
+  float* sP = reinterpret_cast<float*>(smem);                          // [r][d]
+  float* sEt = sP + r * d;                                             // [s][d] (E transposed)
+  __nv_bfloat16* sCR = reinterpret_cast<__nv_bfloat16*>(sEt + d * s);  // per page: C [P][r], R [P][s]
+  double* sMean = reinterpret_cast<double*>(sCR + (size_t)np * P * (r + s));  // [np][r + s]
+  int* sPhys = reinterpret_cast<int*>(sMean + (size_t)np * (r + s));          // [np]
+  const size_t blk_elems = (size_t)P * (r + s);
+  if (tid < npg) {
+    const int ph = p.block_table[(size_t)b * p.max_pages + pg0 + tid];
+    sPhys[tid] = (ph < 0 || ph >= p.num_phys) ? -1 : ph;  // reported by the latent kernel
+  }
+  __syncthreads();
+  // this run's C and R blocks, every copy in flight at once
+  const int c_pieces = P * r * 2 / 16, r_pieces = P * s * 2 / 16;
+  const __nv_bfloat16* clat = static_cast<const __nv_bfloat16*>(p.c_lat);
+  const __nv_bfloat16* rres = static_cast<const __nv_bfloat16*>(p.r_res);
+  for (int i = tid; i < npg * (c_pieces + r_pieces); i += kSumThreads) {
+    const int pi = i / (c_pieces + r_pieces), x = i - pi * (c_pieces + r_pieces);
+    const int ph = sPhys[pi];
+    if (ph < 0) continue;
+    const size_t blk = (size_t)ph * p.Hkv + g;
+    __nv_bfloat16* dst = sCR + (size_t)pi * blk_elems;
+    if (x < c_pieces)
+      cp_async16_cg(dst + x * 8, clat + blk * P * r + x * 8);
+    else
+      cp_async16_cg(dst + (size_t)P * r + (x - c_pieces) * 8, rres + blk * P * s + (x - c_pieces) * 8);
+  }
+  cp_async_commit_group();
+  // the factors meanwhile (fp32, E transposed)
   const __nv_bfloat16* Pm = static_cast<const __nv_bfloat16*>(p.P) + (size_t)g * r * d;
   const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(p.E) + (size_t)g * d * s;
   for (int i = tid; i < r * d; i += kSumThreads) sP[i] = __bfloat162float(Pm[i]);
-  for (int i = tid; i < d * s; i += kSumThreads) sE[i] = __bfloat162float(E[i]);
+  for (int i = tid; i < d * s; i += kSumThreads) {
+    const int x = i / s, q = i - x * s;
+    sEt[q * d + x] = __bfloat162float(E[i]);
+  }
+  cp_async_wait_group<0>();
+  __syncthreads();
+  // column means of every page's valid tokens (fp64, tokens in order)
   const bool swz_on = kc_swizzled(true, d, r);
   const int mc = swz_on ? swz_mask(r) : 0;
-  const __nv_bfloat16* clat = static_cast<const __nv_bfloat16*>(p.c_lat);
-  const __nv_bfloat16* rres = static_cast<const __nv_bfloat16*>(p.r_res);
-  for (int page = pg0; page <= min(last_page, pg0 + kSumPages - 1); ++page) {
-    const int phys = p.block_table[(size_t)b * p.max_pages + page];
-    __syncthreads();  // factors staged / the previous page's sMean consumed
-    if (phys < 0 || phys >= p.num_phys) continue;  // reported by the latent kernel
-    const size_t blk = (size_t)phys * p.Hkv + g;
+  for (int i = tid; i < npg * (r + s); i += kSumThreads) {
+    const int pi = i / (r + s), j = i - pi * (r + s);
+    if (sPhys[pi] < 0) continue;
+    const int page = pg0 + pi;
     const int m = min(L, (page + 1) * P) - page * P;
-    for (int j = tid; j < r + s; j += kSumThreads) {
-      double acc = 0.0;
-      if (j < r) {
-        for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(clat[(blk * P + t) * r + swz(j, t, mc)]);
-      } else {
-        for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(rres[(blk * P + t) * s + (j - r)]);
-      }
-      sMean[j] = acc / (double)m;
+    const __nv_bfloat16* blkp = sCR + (size_t)pi * blk_elems;
+    double acc = 0.0;
+    if (j < r) {
+      for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(blkp[t * r + swz(j, t, mc)]);
+    } else {
+      for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(blkp[(size_t)P * r + t * s + (j - r)]);
     }
-    __syncthreads();
-    for (int x = tid; x < d; x += kSumThreads) {
-      double acc = 0.0;
-      for (int j = 0; j < r; ++j) acc = fma(sMean[j], (double)sP[j * d + x], acc);
-      double acc2 = 0.0;
-      for (int q = 0; q < s; ++q) acc2 = fma(sMean[r + q], (double)sE[x * s + q], acc2);
-      p.summary[blk * d + x] = __double2float_rn(acc + acc2);
-    }
+    sMean[(size_t)pi * (r + s) + j] = acc / (double)m;
+  }
+  __syncthreads();
+  for (int i = tid; i < npg * d; i += kSumThreads) {
+    const int pi = i / d, x = i - pi * d;
+    if (sPhys[pi] < 0) continue;
+    const double* mean = sMean + (size_t)pi * (r + s);
+    double acc = 0.0;
+    for (int j = 0; j < r; ++j) acc = fma(mean[j], (double)sP[j * d + x], acc);
+    double acc2 = 0.0;
+    for (int q = 0; q < s; ++q) acc2 = fma(mean[r + q], (double)sEt[q * d + x], acc2);
+    const size_t blk = (size_t)sPhys[pi] * p.Hkv + g;
+    p.summary[blk * d + x] = __double2float_rn(acc + acc2);
   }
 }
 
@@ -402,7 +447,8 @@ bool prefill_tc_supported(bool bf16, int d, int r, int s) {
   // head_dim 128 only: the shapes the parity tests exercise (64 would take the same code with one
   // K atom per operand, and is left to basiskv_append until it is tested)
   return bf16 && d == 128 && r >= 16 && r <= 128 && r % 16 == 0 && s >= 16 && s <= 64 &&
-         s % 16 == 0 && pf_layout(d, r, s).total + 1024 <= 227 * 1024;
+         s % 16 == 0 && pf_layout(d, r, s).total + 1024 <= 227 * 1024 &&
+         sum_smem_bytes(d, r, s, 16) <= 227 * 1024;
 }
 
 cudaError_t launch_prefill_tc(const AppendParams& p, int num_sms, cudaStream_t st) {
@@ -415,11 +461,12 @@ cudaError_t launch_prefill_tc(const AppendParams& p, int num_sms, cudaStream_t s
   const int split = std::max(1, std::min(ntiles, num_sms / std::max(1, groups)));
   prefill_tc_kernel<<<dim3(split, p.Hkv, p.batch), kPfThreads, smem, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t ssmem = (size_t)(p.r * p.d + p.d * p.s) * sizeof(float) + (size_t)(p.r + p.s) * sizeof(double);
+  const int np = sum_pages(p.page);
+  const size_t ssmem = sum_smem_bytes(p.d, p.r, p.s, p.page);
   if ((e = ensure_smem((const void*)page_summary_kernel, ssmem)) != cudaSuccess) return e;
   // pages touched by n_new tokens starting anywhere inside a page
   const int touched = (p.n_new + p.page - 1) / p.page + 1;
-  page_summary_kernel<<<dim3((touched + kSumPages - 1) / kSumPages, p.Hkv, p.batch), kSumThreads, ssmem, st>>>(p);
+  page_summary_kernel<<<dim3((touched + np - 1) / np, p.Hkv, p.batch), kSumThreads, ssmem, st>>>(p, np);
   return cudaGetLastError();
 }
 

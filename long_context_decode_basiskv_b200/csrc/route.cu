@@ -26,6 +26,12 @@
 //     the lowest page indices; two block scans (ties, kept pages) give every
 //     thread its output positions, so sel is written in ascending page order.
 // The result is the same as sorting by (score descending, page ascending).
+// The G selection CTAs of a KV group run as one thread-block cluster; each
+// ORs its kept pages, with its head's bit, into a head mask per page held in
+// the shared memory of the cluster's first CTA (distributed shared memory),
+// which then writes the group's union list for the attention kernel
+// (union.cuh).  Block tables wider than 8192 pages take a histogram selection
+// whose last CTA per group (an arrival counter) builds the list instead.
 //
 // Per-group routing (group_mode 1 / 2): the score kernel folds the G head
 // scores of a page, which sit on neighbouring lanes after the transpose
@@ -238,14 +244,17 @@ __device__ __forceinline__ void select_union_tail(const RouteParams& p, int b, i
   __syncthreads();
   if (!*s_flag) return;
   union_from_selection(p.sel, p.sel_cnt, p.block_table, p.seq_len[b], b, g, p.Hq, p.Hkv, p.page, p.max_pages,
-                       p.num_phys, p.top_k, p.lists + bg * p.ustride, p.ucount + bg, p.acnt, p.err, masks,
-                       bt_smem, warp_tot);
+                       p.num_phys, p.top_k, p.lists + bg * p.ustride, p.ucount + bg, p.acnt,
+                       (size_t)p.batch * p.Hkv, p.err, masks, bt_smem, warp_tot);
 }
 
-// The selection proper of route_select_kernel (n > top_k + 2 pages).
+// The selection proper of route_select_kernel (n > top_k + 2 pages).  Before
+// it writes the kept pages it waits on the cluster barrier the caller arrived
+// at (the first CTA's masks are zero then) and ORs `hbits` into the mask byte
+// of each kept page in that CTA's shared memory.
 template <int KPT>
 __device__ __forceinline__ void select_rows_reg(const RouteParams& p, const SelRows& rows, int b, int n, int* red,
-                                                int* warp_tot) {
+                                                int* warp_tot, uint32_t* masks, uint32_t hbits) {
   const int tid = threadIdx.x;
   const int kk = p.top_k;
   // thread t holds pages [t * KPT, t * KPT + KPT)
@@ -306,33 +315,71 @@ __device__ __forceinline__ void select_rows_reg(const RouteParams& p, const SelR
   }
   int total;
   int pos = block_exclusive_scan(kept, warp_tot, total);
+  cluster_wait_acquire();
 #pragma unroll
   for (int j = 0; j < KPT; ++j)
-    if (take[j]) put_sel(p, rows, pos++, p0 + j);
+    if (take[j]) {
+      put_sel(p, rows, pos++, p0 + j);
+      red_or_cluster(&masks[(p0 + j) >> 2], hbits << (((p0 + j) & 3) * 8), 0u);
+    }
   for (int i = total + tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, -1);
   if (tid == 0) put_cnt(p, rows, total);
 }
 
+// One CTA per (sequence, query head), or per (sequence, KV group) in the group
+// modes.  The G CTAs of a KV group run as one thread-block cluster: each ORs
+// the pages it kept, with its head's bit, into the head mask per page that the
+// cluster's first CTA holds in shared memory (distributed shared memory), and
+// that CTA writes the group's union list once every CTA's bits are in.
 template <int KPT>
 __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
   __shared__ int red[2 * kSelectWarps];
   __shared__ int warp_tot[32];
-  __shared__ uint32_t s_masks[kSelectThreads * KPT / 4];  // the union's page masks (tail)
-  __shared__ int32_t s_bt[kSelectThreads * KPT];           // the sequence's block-table row (tail)
-  __shared__ int s_flag;
+  __shared__ uint32_t s_masks[kSelectThreads * KPT / 4];  // the group's head masks (first CTA's copy)
+  __shared__ int32_t s_bt[kSelectThreads * KPT];           // the sequence's block-table row (first CTA)
   allow_dependents();  // the union lists' reader may launch; it waits for this grid
   const int b = blockIdx.y, tid = threadIdx.x;
   const int L = p.seq_len[b];
   const int n = max(1, min((L + p.page - 1) / p.page, p.max_pages));
+  const int nu = (L <= 0) ? 0 : n;  // pages of the union list
   const int kk = p.top_k;
+  const int G = p.Hq / p.Hkv;
+  const int g = p.group_mode ? (int)blockIdx.x : (int)blockIdx.x / G;
+  const size_t bg = (size_t)b * p.Hkv + g;
+  const uint32_t crank = cluster_ctarank();
   const SelRows rows = sel_rows(p, blockIdx.x, b);
+  const uint32_t all_heads = (G >= 8) ? 0xffu : ((1u << G) - 1u);
+  const uint32_t hbits = p.group_mode ? all_heads : (1u << (blockIdx.x % G));
+  if (crank == 0) {
+    // the block-table row comes in while the rows are ranked
+    const int32_t* bt_row = p.block_table + (size_t)b * p.max_pages;
+    for (int i = tid; i < nu; i += kSelectThreads) cp_async4(&s_bt[i], bt_row + i);
+    cp_async_commit_group();
+    for (int w = tid; w < (nu + 3) / 4; w += kSelectThreads) s_masks[w] = 0u;
+    cluster_arrive_release();  // the masks are zero from here on
+  } else {
+    cluster_arrive_relaxed();
+  }
   if (n <= kk + 2) {
     for (int i = tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, (i < n) ? i : -1);
     if (tid == 0) put_cnt(p, rows, n);
+    cluster_wait_acquire();
+    for (int pg = tid; pg < nu; pg += kSelectThreads) red_or_cluster(&s_masks[pg >> 2], hbits << ((pg & 3) * 8), 0u);
   } else {
-    select_rows_reg<KPT>(p, rows, b, n, red, warp_tot);
+    select_rows_reg<KPT>(p, rows, b, n, red, warp_tot, s_masks, hbits);
   }
-  select_union_tail(p, b, blockIdx.x, s_masks, s_bt, warp_tot, &s_flag);
+  if (crank != 0) {
+    cluster_arrive_release();  // this CTA's bits are in
+    cluster_wait_acquire();
+    return;
+  }
+  cluster_arrive_relaxed();
+  cluster_wait_acquire();  // every CTA's bits are in the masks
+  cp_async_wait_group<0>();
+  __syncthreads();  // the block-table row is in shared memory
+  if (tid == 0) zero_group_counters(p.acnt, bg, (size_t)p.batch * p.Hkv);  // the attention kernel's counters
+  write_union_list(s_masks, nu, s_bt, L, p.page, p.num_phys, p.lists + bg * p.ustride, p.ucount + bg, p.err,
+                   warp_tot);
 }
 
 // ---------------------------------------------------------------------------
@@ -611,12 +658,22 @@ cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cu
     e = (d == 128) ? launch_score_g<float, 128>(p, G, st) : launch_score_g<float, 64>(p, G, st);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.group_mode ? p.Hkv : p.Hq, p.batch);
-  if (p.max_pages <= kSelectThreads * 8) {
-    route_select_kernel<8><<<grid, kSelectThreads, 0, st>>>(p);
-  } else if (p.max_pages <= kSelectThreads * 16) {
-    route_select_kernel<16><<<grid, kSelectThreads, 0, st>>>(p);
-  } else if (p.max_pages <= kSelectThreads * 32) {
-    route_select_kernel<32><<<grid, kSelectThreads, 0, st>>>(p);
+  if (p.max_pages <= kSelectThreads * 32) {
+    // the G heads of a KV group as one cluster (one CTA per group in the group modes)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.group_mode ? 1 : G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (p.max_pages <= kSelectThreads * 8) return cudaLaunchKernelEx(&cfg, route_select_kernel<8>, p);
+    if (p.max_pages <= kSelectThreads * 16) return cudaLaunchKernelEx(&cfg, route_select_kernel<16>, p);
+    return cudaLaunchKernelEx(&cfg, route_select_kernel<32>, p);
   } else {
     const size_t smem = (size_t)p.max_pages * sizeof(float);
     if ((e = ensure_smem((const void*)route_select_hist_kernel, smem)) != cudaSuccess) return e;

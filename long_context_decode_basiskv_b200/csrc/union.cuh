@@ -23,6 +23,14 @@
 namespace bkv {
 
 constexpr uint32_t kNoPage = 0xffffffu;      // entry id of a page whose block-table entry is out of range
+// The attention kernels keep kGroupCounters int counters per group (the
+// finished splits), in planes of B Hkv ints; whoever writes a group's list
+// sets them to zero.
+constexpr int kGroupCounters = 1;
+__device__ __forceinline__ void zero_group_counters(int32_t* cnt, size_t bg, size_t ngroups) {
+#pragma unroll
+  for (int i = 0; i < kGroupCounters; ++i) cnt[(size_t)i * ngroups + bg] = 0;
+}
 constexpr int kMaxPhysPages = 0xffffff;      // physical page ids must fit the 24 id bits
 
 __host__ __device__ __forceinline__ int union_stride_words(int umax) { return (4 + umax + 3) & ~3; }
@@ -74,14 +82,13 @@ __device__ __forceinline__ void write_union_list(const uint32_t* mask8, int n, c
 // (may be NULL) shared scratch of max_pages words that receives the sequence's
 // block-table row while the selections load.  A selected page outside [0, n)
 // sets BASISKV_DEVERR_SELECTION and is dropped.  Also zeroes the group's
-// attention split counter (acnt) for the attention launch that reads the
-// list, whatever the scratch held before.
+// attention counters (acnt) for the attention launch that reads the list, whatever the scratch held before (`ngroups` = B Hkv).
 __device__ __forceinline__ void union_from_selection(const int32_t* sel, const int32_t* sel_cnt,
                                                      const int32_t* block_table, int L, int b, int g, int Hq,
                                                      int Hkv, int page, int max_pages, int num_phys, int top_k,
                                                      uint32_t* list, uint32_t* ucount, int32_t* acnt,
-                                                     int32_t* err, uint32_t* masks, int32_t* bt_smem,
-                                                     int* warp_tot) {
+                                                     size_t ngroups, int32_t* err, uint32_t* masks,
+                                                     int32_t* bt_smem, int* warp_tot) {
   const int tid = threadIdx.x;
   const int G = Hq / Hkv;
   const int row_len = top_k + 2;
@@ -90,9 +97,7 @@ __device__ __forceinline__ void union_from_selection(const int32_t* sel, const i
   if (n > max_pages) n = max_pages;
   const size_t row0 = (size_t)b * Hq + (size_t)g * G;
   const int32_t* bt_row = block_table + (size_t)b * max_pages;
-  if (tid == 0) {
-    acnt[(size_t)b * Hkv + g] = 0;
-  }
+  if (tid == 0) zero_group_counters(acnt, (size_t)b * Hkv + g, ngroups);
   const int words = (max_pages + 3) / 4;
   for (int i = tid; i < words; i += blockDim.x) masks[i] = 0u;
   if (bt_smem)

@@ -163,13 +163,11 @@ def test_end_to_end(run):
 
 
 def test_step_repeats(run):
-    """A second step on the same inputs selects the same pages and gives the same outputs
-    to within the tolerance (the attention kernel splits a group's tiles among its warps at
-    run time, so the order of its floating-point sums may differ between calls)."""
-    eng, wl = run.eng, run.wl
+    """A second step on the same inputs gives bitwise identical selections and outputs (the
+    split of the attention work depends only on the union sizes)."""
+    eng = run.eng
     s0, c0, o0, y0 = run.outputs
     eng.step()
     torch.cuda.synchronize()
     assert torch.equal(eng.sel, s0) and torch.equal(eng.sel_cnt, c0)
-    assert_close(eng.o_lat.cpu().numpy(), o0.cpu().numpy(), storage_of(wl), "o_lat, second step")
-    assert_close(eng.y.cpu().numpy(), y0.cpu().numpy(), storage_of(wl), "y, second step")
+    assert torch.equal(eng.o_lat, o0) and torch.equal(eng.y, y0)
