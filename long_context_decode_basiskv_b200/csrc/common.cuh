@@ -191,7 +191,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // Global -> shared bulk copy of `bytes` (multiple of 16, both addresses
-// 16-byte aligned), completing on `bar` as transaction bytes.  No multicast.
+// 16-byte aligned), completing on `bar` as transaction bytes; the data lands in this CTA only.
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes,
                                          uint64_t* bar) {
   asm volatile(

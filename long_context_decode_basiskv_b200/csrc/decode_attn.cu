@@ -21,8 +21,8 @@
 //   * attn_mma_kernel (bf16 with the swizzled K/C layout, the main path): four
 //     warps per CTA take the share's 16-token tiles round-robin, each with its
 //     own ring of bulk copies (cp.async.bulk, mbarrier completion, bounded
-//     waits, no multicast), and run all G heads of the group on the tensor
-//     cores (mma.sync m16n8k16); the warps' states are folded in warp order.
+//     waits), and run all G heads of the group on the tensor cores
+//     (mma.sync m16n8k16); the warps' states are folded in warp order.
 //     The split of the work depends only on the union sizes, so the output is
 //     reproducible.
 //   * attn_kernel (fp32 and shapes without the swizzled layout): warp 0
@@ -538,8 +538,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // kernel), so the splits of all groups hold about the same number of tiles;
 // split s of a group's ns takes an equal contiguous share of the group's
 // union list.  The four warps take the share's tiles round-robin, each with
-// its own ring of 1-D bulk copies (mbarrier completion, bounded waits, no
-// multicast), and run all G heads of the group on the tensor cores
+// its own ring of 1-D bulk copies (mbarrier completion, bounded waits), and
+// run all G heads of the group on the tensor cores
 // (mma.sync m16n8k16).  At the end the warps' states are folded in warp order
 // into the CTA's partial result; the last CTA of the group merges the
 // group's partials into o_lat.  The split of the work depends only on the

@@ -13,7 +13,7 @@
 // image the MMA reads, and the k-chunks of an m-tile are consecutive, so each
 // CTA streams one contiguous region with 1-D bulk copies.
 //
-// Per CTA: warp 0 streams the 16 KB tiles of Gt (cp.async.bulk, no multicast)
+// Per CTA: warp 0 streams the 16 KB tiles of Gt (cp.async.bulk into this CTA only)
 // into a ring of 4-8 stages and one of its threads issues the
 // tcgen05.mma instructions, refilling each stage one iteration after its MMAs
 // were committed; warps 1-4 prefetch the matching slices of o with cp.async,
