@@ -17,6 +17,9 @@
  *                        Value latents (rank-r output per head)
  *   basiskv_out_proj     (step 5)   y = sum_h o_h G_h through the fused factor
  *
+ * A step whose inputs and output live in page-locked host memory brings the
+ * inputs in with basiskv_copy and lets basiskv_out_proj store y on the host.
+ *
  * Method: "BasisKV: Value Latents for Communication and Key Routing"
  * (weekinpapers.com/paper/2611.02583v1, Abstract) and the kongchang.com
  * explainer of it (sections on binding the Value latent to the output
@@ -63,7 +66,7 @@ extern "C" {
 /* 1: append, route, decode_attn, out_proj and their helpers;
  * 2: adds basiskv_route_group and basiskv_prefill;
  * 3: decode_attn accepts sel = sel_cnt = NULL (the routing call's selection). */
-#define BASISKV_ABI_VERSION 3
+#define BASISKV_ABI_VERSION 4
 
 typedef enum {
   BASISKV_OK = 0,
@@ -297,6 +300,12 @@ BASISKV_API basiskv_status basiskv_decode_attn_noalloc(const basiskv_config* cfg
 /*
  * Step 5.  y[b] = sum_h o_lat[b][h] G_h (fp32 [batch][hidden]) with G read from
  * factors->Gt.  The full Value width is never formed.  workspace as above.
+ * y may be device memory or page-locked host memory that the runtime has
+ * mapped into the device's address space (cudaHostAlloc / cudaMallocHost, or
+ * cudaHostRegister with mapping, under unified addressing): the kernel then
+ * stores the result straight into host memory, readable once the stream has
+ * been synchronised.  Any other y (pageable host memory) returns
+ * BASISKV_ERR_INVALID_ARG and launches nothing.
  */
 BASISKV_API basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors* factors,
                                 const float* o_lat, int32_t batch, float* y, void* workspace,
@@ -311,6 +320,20 @@ BASISKV_API basiskv_status basiskv_out_proj(const basiskv_config* cfg, const bas
  */
 BASISKV_API basiskv_status basiskv_fuse_out_factor(const basiskv_config* cfg, const void* Bf,
                                        const void* W_O, void* Gt, void* stream);
+
+/*
+ * Copies `bytes` from src to dst on `stream` with a kernel (the SMs' own loads
+ * and stores, no copy engine): either side may be device memory or page-locked
+ * host memory mapped into the device's address space, as for basiskv_out_proj's
+ * y.  Meant for a decode step's small inputs (q, k_new, v_new: about 100 KB),
+ * where a copy-engine transfer captured in a CUDA graph costs several times the
+ * bytes' wire time.  Both pointers 16-byte aligned, ranges not overlapping;
+ * host memory that is not mapped, a NULL pointer with bytes > 0 or a
+ * misaligned pointer returns BASISKV_ERR_INVALID_ARG and launches nothing.
+ * Asynchronous: the caller keeps src unchanged and does not read dst until the
+ * stream has passed the copy.  bytes = 0 does nothing.
+ */
+BASISKV_API basiskv_status basiskv_copy(void* dst, const void* src, size_t bytes, void* stream);
 
 /* Workspace bytes needed by route / decode_attn / out_proj for this shape. */
 BASISKV_API size_t basiskv_workspace_bytes(const basiskv_config* cfg, int32_t batch, int32_t max_pages);

@@ -27,6 +27,7 @@ SYMBOLS = [
     "basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
     "basiskv_fuse_out_factor", "basiskv_workspace_bytes", "basiskv_status_string",
     "basiskv_abi_version", "basiskv_decode_attn_noalloc", "basiskv_route_group", "basiskv_prefill",
+    "basiskv_copy",
 ]
 
 
@@ -70,6 +71,7 @@ def lib():
     L.basiskv_out_proj.argtypes = [pc, pf, vp, i32, vp, vp, sz, vp]
     L.basiskv_decode_attn_noalloc.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, vp]
     L.basiskv_fuse_out_factor.argtypes = [pc, vp, vp, vp, vp]
+    L.basiskv_copy.argtypes = [vp, vp, sz, vp]
     L.basiskv_workspace_bytes.argtypes = [pc, i32, i32]
     L.basiskv_workspace_bytes.restype = sz
     L.basiskv_status_string.argtypes = [i32]
@@ -77,7 +79,7 @@ def lib():
     L.basiskv_abi_version.argtypes = []
     for name in ["basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
                  "basiskv_fuse_out_factor", "basiskv_abi_version", "basiskv_decode_attn_noalloc",
-                 "basiskv_route_group", "basiskv_prefill"]:
+                 "basiskv_route_group", "basiskv_prefill", "basiskv_copy"]:
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -131,6 +133,22 @@ def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
         raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _need_reachable(t: torch.Tensor, name: str, dtype=None, shape=None):
+    """_need, but a page-locked CPU tensor is also accepted (the kernels reach it
+    through the runtime's mapping of pinned host memory)."""
+    if isinstance(t, torch.Tensor) and not t.is_cuda:
+        if not t.is_pinned():
+            raise ValueError(f"{name} must be a CUDA tensor or a pinned CPU tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+        if shape is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+        return
+    _need(t, name, dtype, shape)
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -278,10 +296,21 @@ def out_proj(cfg: Config, f: Factors, o_lat: torch.Tensor, y: torch.Tensor, ws: 
              stream=None):
     B = o_lat.shape[0]
     _need(o_lat, "o_lat", torch.float32, (B, cfg.num_q_heads, cfg.rank_v))
-    _need(y, "y", torch.float32, (B, cfg.hidden))
+    _need_reachable(y, "y", torch.float32, (B, cfg.hidden))  # device, or pinned host: stored there directly
     _need(ws, "workspace", torch.uint8)
     _check(lib().basiskv_out_proj(ctypes.byref(cfg.c()), ctypes.byref(f.c()), _ptr(o_lat), B, _ptr(y),
                                   _ptr(ws), ws.numel(), _stream(stream)), "basiskv_out_proj")
+
+
+def copy(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    """dst <- src (same dtype and element count) by a kernel: either may be a CUDA tensor
+    or a pinned CPU tensor (basiskv_copy)."""
+    _need_reachable(dst, "dst")
+    _need_reachable(src, "src", dst.dtype)
+    if dst.numel() != src.numel():
+        raise ValueError(f"copy: {src.numel()} elements into {dst.numel()}")
+    _check(lib().basiskv_copy(_ptr(dst), _ptr(src), src.numel() * src.element_size(), _stream(stream)),
+           "basiskv_copy")
 
 
 def decode_attn_noalloc(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor,

@@ -49,6 +49,20 @@ static basiskv_status check_cache(const basiskv_config* c, const basiskv_cache* 
   return BASISKV_OK;
 }
 
+// The address under which kernels reach `p`: p itself for device or managed
+// memory, the mapping of page-locked host memory allocated or registered with
+// the runtime; NULL for anything else (pageable host memory, unknown pointers).
+static void* device_view(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();  // the error is not sticky: clear it so a later check does not see it
+    return nullptr;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return const_cast<void*>(p);
+  if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+  return nullptr;
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -246,6 +260,8 @@ basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors
   if (batch == 0) return BASISKV_OK;
   if (!f || !f->Gt || !o_lat || !y || batch < 0) return BASISKV_ERR_INVALID_ARG;
   if (!aligned16(f->Gt) || !aligned16(o_lat) || !aligned16(y)) return BASISKV_ERR_INVALID_ARG;
+  y = static_cast<float*>(device_view(y));  // device memory, or page-locked host memory the kernel writes
+  if (!y || !aligned16(y)) return BASISKV_ERR_INVALID_ARG;
   (void)ws;
   (void)ws_bytes;
   const int K = cfg->num_q_heads * cfg->rank_v;
@@ -256,6 +272,18 @@ basiskv_status basiskv_out_proj(const basiskv_config* cfg, const basiskv_factors
                                           (cudaStream_t)stream));
   OutProjParams p{o_lat, f->Gt, y, batch, K, cfg->hidden};
   return cuda_status(launch_out_proj_gemv(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
+}
+
+basiskv_status basiskv_copy(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return BASISKV_OK;
+  if (!dst || !src) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(dst) || !aligned16(src)) return BASISKV_ERR_INVALID_ARG;
+  void* d = device_view(dst);
+  const void* s = device_view(src);
+  if (!d || !s || !aligned16(d) || !aligned16(s)) return BASISKV_ERR_INVALID_ARG;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(d), b = reinterpret_cast<uintptr_t>(s);
+  if (a < b + bytes && b < a + bytes) return BASISKV_ERR_INVALID_ARG;  // overlapping ranges
+  return cuda_status(launch_copy(d, s, bytes, num_sms(), (cudaStream_t)stream));
 }
 
 basiskv_status basiskv_fuse_out_factor(const basiskv_config* cfg, const void* Bf, const void* W_O,

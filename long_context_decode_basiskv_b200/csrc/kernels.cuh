@@ -136,6 +136,9 @@ cudaError_t launch_out_proj_mma(const float* o, const void* Gt, float* y, int ba
 cudaError_t launch_out_proj_tc(const float* o, const void* Gt, float* y, int32_t* err, int batch, int K, int hidden,
                                int num_sms, cudaStream_t st);
 
+// bytes from src to dst by the SMs (either side device memory or mapped host memory)
+cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t st);
+
 struct FuseParams {
   const void* Bf;
   const void* W_O;

@@ -110,8 +110,10 @@ class DecodeEngine:
         sel, cnt = (None, None) if from_route else (self.sel, self.sel_cnt)
         bk.decode_attn(self.cfg, self.cache, self.q, sel, cnt, self.o_lat, self.ws, self.err, stream)
 
-    def out_proj(self, stream=None):
-        bk.out_proj(self.cfg, self.factors, self.o_lat, self.y, self.ws, stream)
+    def out_proj(self, stream=None, y=None):
+        """y defaults to the engine's device tensor; a pinned CPU tensor of its shape
+        receives the result straight from the kernel."""
+        bk.out_proj(self.cfg, self.factors, self.o_lat, self.y if y is None else y, self.ws, stream)
 
     def append_route(self, stream=None):
         """Append (on a forked stream) concurrently with route, then join.
@@ -131,12 +133,13 @@ class DecodeEngine:
         self.route(stream=main)
         main.wait_event(self._join)
 
-    def step(self, stream=None):
-        """One decode step: (append || route) -> decode_attn -> out_proj."""
+    def step(self, stream=None, y=None):
+        """One decode step: (append || route) -> decode_attn -> out_proj (into y, by
+        default the engine's device tensor)."""
         self.append_route(stream)
         self.decode_attn(stream)
-        self.out_proj(stream)
-        return self.y
+        self.out_proj(stream, y)
+        return self.y if y is None else y
 
     def graph_step(self):
         """step() replayed from a CUDA graph captured on first use (the inputs are
@@ -155,9 +158,10 @@ class DecodeEngine:
         return self.y
 
     def graph_step_host(self, host_in: torch.Tensor, host_y: torch.Tensor):
-        """One decode step with host buffers, replayed from one CUDA graph: the copy of the
-        step's inputs from `host_in` (pinned, input_buffer()'s layout and dtype), the four
-        calls, and the copy of y into `host_y` (pinned, y's shape and dtype).  The graph is
+        """One decode step with host buffers, replayed from one CUDA graph: the step's
+        inputs come from `host_in` (pinned, input_buffer()'s layout and dtype) through
+        basiskv_copy, then the four calls, the out-projection storing y straight into
+        `host_y` (pinned, y's shape and dtype); no copy-engine transfer.  The graph is
         captured on the first call for these two buffers; the caller refills host_in before
         a call and reads host_y once the current stream is synchronised."""
         if not (host_in.is_pinned() and host_y.is_pinned()):
@@ -175,9 +179,8 @@ class DecodeEngine:
             torch.cuda.current_stream(self.device).wait_stream(side)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=side):
-                self._inbuf.copy_(host_in, non_blocking=True)
-                self.step()
-                host_y.copy_(self.y, non_blocking=True)
+                bk.copy(self._inbuf, host_in)
+                self.step(y=host_y)
             self._io_graph, self._io_key = g, key
         self._io_graph.replay()
         return host_y

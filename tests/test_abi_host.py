@@ -58,7 +58,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.basiskv_abi_version() == 3
+    assert L.basiskv_abi_version() == 4
     assert L.basiskv_status_string(0) == b"ok"
     assert L.basiskv_status_string(4).startswith(b"workspace")
     assert L.basiskv_status_string(99) == b"unknown status"
