@@ -157,10 +157,7 @@ typedef struct {
  * the raw key is stored as given.  Then every touched page's summary is
  * recomputed over its valid tokens: S = mean(C) P_g + mean(R) E_g^T, rounded
  * to fp32.  n_new = 1 is the decode step; larger n_new is prefill.
- * With n_new = 1 and factors->Gt set, the call also starts bringing Gt into
- * L2 (a prefetch, no result depends on it), so the step's basiskv_out_proj
- * finds it cached; the sparse-attention and routing streams are read with an
- * evict-first L2 policy and do not displace it.
+ * factors->Gt is not read (it may be NULL).
  * err_flag (device int32) may not be NULL.
  */
 BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* cache,

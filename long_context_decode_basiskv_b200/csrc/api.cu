@@ -171,16 +171,10 @@ basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* ca
     return BASISKV_ERR_INVALID_ARG;
   if (!aligned16(f->A) || !aligned16(f->P) || !aligned16(f->E)) return BASISKV_ERR_INVALID_ARG;
   if ((long long)n_new > (long long)cache->max_pages * cfg->page_size) return BASISKV_ERR_INVALID_ARG;
-  AppendParams p{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
-                 cache->summary, cache->block_table, cache->seq_len, err_flag,
-                 batch, n_new, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
-                 cfg->page_size, cache->max_pages, cache->num_phys_pages, nullptr, 0};
-  // the decode step's out-projection reads the whole fused factor: start bringing it into L2 now
-  const size_t gt_bytes = (size_t)cfg->hidden * cfg->num_q_heads * cfg->rank_v * esize(cfg);
-  if (n_new == 1 && f->Gt && aligned16(f->Gt) && gt_bytes % 16 == 0) {
-    p.warm = f->Gt;
-    p.warm_bytes = gt_bytes;
-  }
+  const AppendParams p{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
+                       cache->summary, cache->block_table, cache->seq_len, err_flag,
+                       batch, n_new, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
+                       cfg->page_size, cache->max_pages, cache->num_phys_pages};
   return cuda_status(launch_append(p, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream));
 }
 
@@ -201,7 +195,7 @@ basiskv_status basiskv_prefill(const basiskv_config* cfg, const basiskv_cache* c
   const AppendParams p{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
                        cache->summary, cache->block_table, cache->seq_len, err_flag,
                        batch, n_new, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
-                       cfg->page_size, cache->max_pages, cache->num_phys_pages, nullptr, 0};
+                       cfg->page_size, cache->max_pages, cache->num_phys_pages};
   return cuda_status(launch_prefill_tc(p, num_sms(), (cudaStream_t)stream));
 }
 

@@ -237,14 +237,6 @@ __global__ void __launch_bounds__(kDecThreads) append_decode_kernel(AppendParams
 
   const size_t blk = (size_t)phys * p.Hkv + g;
   const size_t row = (size_t)b * p.Hkv + g;  // n_new == 1
-  if (p.warm && tid == 0) {
-    // this CTA's share of the bytes to warm in L2, in 64 KB requests
-    const size_t ctas = (size_t)gridDim.x * gridDim.y, me = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-    const size_t share = ((p.warm_bytes / 16 + ctas - 1) / ctas) * 16;
-    const size_t lo = me * share, hi = min(p.warm_bytes, lo + share);
-    for (size_t o = lo; o < hi; o += 65536)
-      prefetch_l2(static_cast<const char*>(p.warm) + o, (uint32_t)min((size_t)65536, hi - o));
-  }
   T* kdst = static_cast<T*>(p.k_raw) + blk * P * d;
   T* cdst = static_cast<T*>(p.c_lat) + blk * P * r;
   T* rdst = static_cast<T*>(p.r_res) + blk * P * s;

@@ -212,18 +212,12 @@ __device__ __forceinline__ void bulk_g2s_hint(void* smem_dst, const void* gmem_s
 }
 
 // L2 policy for data read once: its lines are the first to be replaced, so
-// data of normal priority (the out-projection factor, warmed earlier in the
-// step) stays cached while such a stream passes through.
+// data of normal priority (union lists, split partials, the out-projection
+// factor where it fits) stays cached while such a stream passes through.
 __device__ __forceinline__ uint64_t l2_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
-}
-
-// Bring `bytes` (a multiple of 16, 16-byte aligned) at `src` into L2 without
-// waiting for it.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 

@@ -19,8 +19,6 @@ struct AppendParams {
   const int32_t* seq_len;
   int32_t* err;
   int batch, n_new, Hkv, d, r, s, page, max_pages, num_phys;
-  const void* warm;   // optional: bytes to bring into L2 during a decode-step append (the fused factor)
-  size_t warm_bytes;  // a multiple of 16
 };
 cudaError_t launch_append(const AppendParams& p, bool bf16, cudaStream_t st);
 // many tokens per sequence on the tensor cores (bf16 only), then the touched pages' summaries
