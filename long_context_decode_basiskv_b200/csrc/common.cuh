@@ -264,10 +264,12 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 __device__ __forceinline__ void cluster_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void red_or_cluster(uint32_t* local, uint32_t v, uint32_t rank) {
-  uint32_t remote;
+// The word at `local`'s offset in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t ld_shared_cluster(const uint32_t* local, uint32_t rank) {
+  uint32_t remote, v;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("red.shared::cluster.or.b32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
 }
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }
 

@@ -248,13 +248,12 @@ __device__ __forceinline__ void select_union_tail(const RouteParams& p, int b, i
                        (size_t)p.batch * p.Hkv, p.err, masks, bt_smem, warp_tot);
 }
 
-// The selection proper of route_select_kernel (n > top_k + 2 pages).  Before
-// it writes the kept pages it waits on the cluster barrier the caller arrived
-// at (the first CTA's masks are zero then) and ORs `hbits` into the mask byte
-// of each kept page in that CTA's shared memory.
+// The selection proper of route_select_kernel (n > top_k + 2 pages): writes
+// the CTA's sel rows and returns this thread's kept pages as bits (bit j:
+// page tid KPT + j).
 template <int KPT>
-__device__ __forceinline__ void select_rows_reg(const RouteParams& p, const SelRows& rows, int b, int n, int* red,
-                                                int* warp_tot, uint32_t* masks, uint32_t hbits) {
+__device__ __forceinline__ uint32_t select_rows_reg(const RouteParams& p, const SelRows& rows, int n, int* red,
+                                                    int* warp_tot) {
   const int tid = threadIdx.x;
   const int kk = p.top_k;
   // thread t holds pages [t * KPT, t * KPT + KPT)
@@ -272,6 +271,7 @@ __device__ __forceinline__ void select_rows_reg(const RouteParams& p, const SelR
     for (int j = 0; j < KPT; ++j) c += key[j] >= t;
     return c;
   };
+  // T: the largest key with at least k candidate keys >= T, bit by bit
   int phase = 0;
   uint32_t T = 0;
   bool exact = false;
@@ -286,57 +286,55 @@ __device__ __forceinline__ void select_rows_reg(const RouteParams& p, const SelR
       }
     }
   }
-  int keep_eq;
-  if (exact) {
-    T -= 1;  // keep key > T; no ties (at least one bit of T was set)
-    keep_eq = 0;
-  } else {
-    keep_eq = kk - ((T == 0xffffffffu) ? 0 : block_total(count_ge(T + 1), red, phase));
-  }
-  // ties at T before this thread's pages (page order), then kept pages before them
-  int ties = 0;
+  // Kept: pages 0 and n - 1, keys above Tk, and the first keep_eq keys equal
+  // to Tk in page order.  Exactly k keys are >= T when `exact`: keep those
+  // (Tk = T - 1, no key equal to Tk is kept).  Otherwise T is the k-th largest
+  // key and the keys equal to it fill what the larger ones leave.  One scan
+  // counts both classes (above | equal << 16) before each thread.
+  const uint32_t Tk = exact ? T - 1 : T;
+  int above = 0, equal = 0;
 #pragma unroll
-  for (int j = 0; j < KPT; ++j) ties += key[j] != 0u && key[j] == T;
+  for (int j = 0; j < KPT; ++j) {
+    const int pg = p0 + j;
+    above += (pg == 0 || pg == n - 1 || key[j] > Tk) && pg < n;
+    equal += key[j] != 0u && key[j] == Tk;
+  }
   int tot;
-  const int tie0 = block_exclusive_scan(ties, warp_tot, tot);
-  bool take[KPT];
-  int kept = 0;
-  {
-    int tr = tie0;
+  const int before = block_exclusive_scan(above | (equal << 16), warp_tot, tot);
+  const int above_tot = tot & 0xffff, equal_tot = tot >> 16;
+  const int keep_eq = exact ? 0 : kk - (above_tot - 2);  // pages 0 and n - 1 are counted in above_tot
+  const int eq_before = before >> 16;
+  int pos = (before & 0xffff) + min(eq_before, keep_eq);
+  int tie = eq_before;
+  uint32_t bits = 0;
 #pragma unroll
-    for (int j = 0; j < KPT; ++j) {
-      const int pg = p0 + j;
-      const bool tie = key[j] != 0u && key[j] == T;
-      take[j] = pg == 0 || pg == n - 1 || key[j] > T || (tie && tr < keep_eq);
-      take[j] = take[j] && pg < n;
-      tr += tie;
-      kept += take[j];
+  for (int j = 0; j < KPT; ++j) {
+    const int pg = p0 + j;
+    bool take = (pg == 0 || pg == n - 1 || key[j] > Tk) && pg < n;
+    if (key[j] != 0u && key[j] == Tk) take = tie++ < keep_eq;
+    if (take) {
+      put_sel(p, rows, pos++, pg);
+      bits |= 1u << j;
     }
   }
-  int total;
-  int pos = block_exclusive_scan(kept, warp_tot, total);
-  cluster_wait_acquire();
-#pragma unroll
-  for (int j = 0; j < KPT; ++j)
-    if (take[j]) {
-      put_sel(p, rows, pos++, p0 + j);
-      red_or_cluster(&masks[(p0 + j) >> 2], hbits << (((p0 + j) & 3) * 8), 0u);
-    }
+  const int total = above_tot + min(equal_tot, keep_eq);
   for (int i = total + tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, -1);
   if (tid == 0) put_cnt(p, rows, total);
+  return bits;
 }
 
 // One CTA per (sequence, query head), or per (sequence, KV group) in the group
-// modes.  The G CTAs of a KV group run as one thread-block cluster: each ORs
-// the pages it kept, with its head's bit, into the head mask per page that the
-// cluster's first CTA holds in shared memory (distributed shared memory), and
-// that CTA writes the group's union list once every CTA's bits are in.
+// modes.  The G CTAs of a KV group run as one thread-block cluster: each keeps
+// its head's kept pages as bits in its own shared memory, and after a cluster
+// barrier the first CTA reads the others' bits (distributed shared memory),
+// forms the head mask of every page and writes the group's union list.
 template <int KPT>
 __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
   __shared__ int red[2 * kSelectWarps];
   __shared__ int warp_tot[32];
-  __shared__ uint32_t s_masks[kSelectThreads * KPT / 4];  // the group's head masks (first CTA's copy)
-  __shared__ int32_t s_bt[kSelectThreads * KPT];           // the sequence's block-table row (first CTA)
+  __shared__ uint32_t s_take[kSelectThreads];               // this CTA's kept pages, KPT bits per thread
+  __shared__ uint32_t s_masks[kSelectThreads * KPT / 4];    // the group's head masks (first CTA)
+  __shared__ int32_t s_bt[kSelectThreads * KPT];            // the sequence's block-table row (first CTA)
   allow_dependents();  // the union lists' reader may launch; it waits for this grid
   const int b = blockIdx.y, tid = threadIdx.x;
   const int L = p.seq_len[b];
@@ -346,40 +344,64 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParam
   const int G = p.Hq / p.Hkv;
   const int g = p.group_mode ? (int)blockIdx.x : (int)blockIdx.x / G;
   const size_t bg = (size_t)b * p.Hkv + g;
-  const uint32_t crank = cluster_ctarank();
+  const uint32_t crank = cluster_ctarank();  // the head within the group (per-head mode)
+  const int csize = p.group_mode ? 1 : G;
   const SelRows rows = sel_rows(p, blockIdx.x, b);
-  const uint32_t all_heads = (G >= 8) ? 0xffu : ((1u << G) - 1u);
-  const uint32_t hbits = p.group_mode ? all_heads : (1u << (blockIdx.x % G));
+  const int p0 = tid * KPT;
   if (crank == 0) {
-    // the block-table row comes in while the rows are ranked
+    // this thread's block-table entries come in while the rows are ranked
     const int32_t* bt_row = p.block_table + (size_t)b * p.max_pages;
-    for (int i = tid; i < nu; i += kSelectThreads) cp_async4(&s_bt[i], bt_row + i);
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (p0 + j < nu) cp_async4(&s_bt[p0 + j], bt_row + p0 + j);
     cp_async_commit_group();
-    for (int w = tid; w < (nu + 3) / 4; w += kSelectThreads) s_masks[w] = 0u;
-    cluster_arrive_release();  // the masks are zero from here on
-  } else {
-    cluster_arrive_relaxed();
   }
+  uint32_t take;
   if (n <= kk + 2) {
     for (int i = tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, (i < n) ? i : -1);
     if (tid == 0) put_cnt(p, rows, n);
-    cluster_wait_acquire();
-    for (int pg = tid; pg < nu; pg += kSelectThreads) red_or_cluster(&s_masks[pg >> 2], hbits << ((pg & 3) * 8), 0u);
+    const int m = min(KPT, max(0, n - p0));  // every page is kept
+    take = (m >= 32) ? 0xffffffffu : ((1u << m) - 1u);
   } else {
-    select_rows_reg<KPT>(p, rows, b, n, red, warp_tot, s_masks, hbits);
+    take = select_rows_reg<KPT>(p, rows, n, red, warp_tot);
   }
+  s_take[tid] = take;
+  cluster_arrive_release();  // this CTA's kept pages are in its shared memory
+  cluster_wait_acquire();
   if (crank != 0) {
-    cluster_arrive_release();  // this CTA's bits are in
+    cluster_arrive_relaxed();  // the first CTA arrives here once it has read s_take: stay until then
     cluster_wait_acquire();
     return;
   }
-  cluster_arrive_relaxed();
-  cluster_wait_acquire();  // every CTA's bits are in the masks
-  cp_async_wait_group<0>();
-  __syncthreads();  // the block-table row is in shared memory
+  // head masks of this thread's pages: bit r from cluster CTA r (head g G + r)
+  uint32_t tk[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) tk[r] = (r == 0) ? take : (r < csize ? ld_shared_cluster(&s_take[tid], r) : 0u);
+  const uint32_t all_heads = (G >= 8) ? 0xffu : ((1u << G) - 1u);
+#pragma unroll
+  for (int w = 0; w < KPT / 4; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = 4 * w + q;
+      uint32_t m = 0;
+      if (p.group_mode) {
+        m = ((take >> j) & 1u) ? all_heads : 0u;
+      } else {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) m |= ((tk[r] >> j) & 1u) << r;
+      }
+      word |= m << (8 * q);
+    }
+    s_masks[p0 / 4 + w] = word;
+  }
+  cluster_arrive_relaxed();  // the other CTAs' bits are read: they may exit
+  cp_async_wait_group<0>();  // this thread's block-table entries
   if (tid == 0) zero_group_counters(p.acnt, bg, (size_t)p.batch * p.Hkv);  // the attention kernel's counters
-  write_union_list(s_masks, nu, s_bt, L, p.page, p.num_phys, p.lists + bg * p.ustride, p.ucount + bg, p.err,
-                   warp_tot);
+  // each thread lists its own pages (masks and block-table entries it wrote itself)
+  write_union_list_range(s_masks, min(nu, p0), min(nu, p0 + KPT), nu, s_bt, L, p.page, p.num_phys,
+                         p.lists + bg * p.ustride, p.ucount + bg, p.err, warp_tot);
+  cluster_wait_acquire();
 }
 
 // ---------------------------------------------------------------------------

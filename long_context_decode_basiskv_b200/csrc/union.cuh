@@ -35,20 +35,23 @@ constexpr int kMaxPhysPages = 0xffffff;      // physical page ids must fit the 2
 
 __host__ __device__ __forceinline__ int union_stride_words(int umax) { return (4 + umax + 3) & ~3; }
 
-// All threads of the block call this.  `mask8` holds one byte per logical page
-// 0 .. n-1 of the sequence (packed four to a word; nonzero = selected by the
-// heads whose bits are set).  Writes the group's list in ascending page order.
-// `bt_row` is the sequence's block-table row (shared or global memory); a page
-// whose entry is outside [0, num_phys) is stored as kNoPage and sets the error
-// flag.  `L` is the sequence length (the last page may be partial).  The entry
-// count also goes to *ucount, the group's slot of a compact [B][Hkv] array
-// from which the attention kernel shares its CTAs out among the groups.
-__device__ __forceinline__ void write_union_list(const uint32_t* mask8, int n, const int32_t* bt_row, int L,
-                                                 int page, int num_phys, uint32_t* list, uint32_t* ucount,
-                                                 int32_t* err, int* warp_tot) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int per = (n + nthr - 1) / nthr;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
+// All threads of the block call this, each for its pages [lo, hi) (the
+// threads' ranges ascend with the thread index and cover 0 .. n-1).  `mask8`
+// holds one byte per logical page of the sequence (packed four to a word;
+// nonzero = selected by the heads whose bits are set).  Writes the group's
+// list in ascending page order.  `bt_row` is the sequence's block-table row
+// (shared or global memory); a page whose entry is outside [0, num_phys) is
+// stored as kNoPage and sets the error flag.  `L` is the sequence length (the
+// last page may be partial).  The entry count also goes to *ucount, the
+// group's slot of a compact [B][Hkv] array from which the attention kernel
+// shares its CTAs out among the groups.  A thread's own mask bytes and
+// block-table entries need no barrier before the call; thread 0 reads page
+// n-1's byte after the call's first barrier.
+__device__ __forceinline__ void write_union_list_range(const uint32_t* mask8, int lo, int hi, int n,
+                                                       const int32_t* bt_row, int L, int page, int num_phys,
+                                                       uint32_t* list, uint32_t* ucount, int32_t* err,
+                                                       int* warp_tot) {
+  const int tid = threadIdx.x;
   int c = 0;
   for (int pg = lo; pg < hi; ++pg) c += ((mask8[pg >> 2] >> ((pg & 3) * 8)) & 0xffu) ? 1 : 0;
   int tot;
@@ -73,6 +76,16 @@ __device__ __forceinline__ void write_union_list(const uint32_t* mask8, int n, c
     *ucount = (uint32_t)tot;  // the same count, in the compact per-group array
     if (n < 1 || !((mask8[(n - 1) >> 2] >> (((n - 1) & 3) * 8)) & 0xffu)) list[1] = (uint32_t)page;
   }
+}
+
+// write_union_list_range with the pages split evenly over the block's threads.
+__device__ __forceinline__ void write_union_list(const uint32_t* mask8, int n, const int32_t* bt_row, int L,
+                                                 int page, int num_phys, uint32_t* list, uint32_t* ucount,
+                                                 int32_t* err, int* warp_tot) {
+  const int nthr = blockDim.x;
+  const int per = (n + nthr - 1) / nthr;
+  const int lo = min(n, (int)threadIdx.x * per), hi = min(n, lo + per);
+  write_union_list_range(mask8, lo, hi, n, bt_row, L, page, num_phys, list, ucount, err, warp_tot);
 }
 
 // The union list of group (b, g) from the G heads' selection rows: sel
