@@ -48,7 +48,8 @@ static size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 // shared memory of the tensor-core kernel: rings, their barriers, the chunk queue's barriers
 static size_t mma_smem_bytes(int d, int r, int slots, int G) {
   const size_t stage = ((size_t)kTile * (d + r) * 2 + 127) & ~(size_t)127;
-  return (size_t)kMmaWarps * slots * (stage + 8) + (size_t)G * (r + 2) * 4;  // + the CTA's result
+  (void)G;  // the warps' states reuse the first stage of each ring: G (r + 2) floats fit in a 16-row stage
+  return (size_t)kMmaWarps * slots * (stage + 8);
 }
 // ... and of the CUDA-core kernel: ring and full / empty barriers
 static size_t core_smem_bytes(int d, int r, int esize) {
@@ -135,6 +136,7 @@ __device__ __forceinline__ void assign_cta(const AttnParams& p, int c, int* warp
       s_asg[1] = c - cg;
       s_asg[2] = cn - cg;
       s_asg[3] = cg;
+      s_asg[4] = (int)min(__ldcg(p.ucount + g), (uint32_t)p.umax);  // the group's union entries
     }
     P = pn;
   }
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   __shared__ uint32_t meta[kStages];  // head mask | valid tokens << 8 of the tile in each stage
   __shared__ int s_last, s_fail, s_issued, s_consumed;
   __shared__ int warp_tot[32];
-  __shared__ int s_asg[4];
+  __shared__ int s_asg[5];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.r;
   const uint32_t k_bytes = kTile * D * sizeof(T);
@@ -344,8 +346,7 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
   }
 
   const uint32_t* list = p.lists + (size_t)bg * p.ustride;
-  const int U = min((int)__ldcg(list), p.umax);
-  const int tail_valid = (int)__ldcg(list + 1);
+  const int U = s_asg[4];  // list[0], as the compact count array holds it
   const int eps = (U + ns - 1) / ns;
   const int e0 = split * eps;
   const int nent = max(0, min(U, e0 + eps) - e0);
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(32 * (G + 1)) attn_kernel(AttnParams p) {
       if (cb + lane < nent) {
         const int e = e0 + cb + lane;
         my_en = __ldcg(list + 4 + e);
-        my_valid = (e == U - 1) ? tail_valid : p.page;
+        my_valid = (e == U - 1) ? (int)__ldcg(list + 1) : p.page;
       }
       const int t_end = min(nent, cb + 32) * p.tpp;
       for (; t < t_end; ++t) {
@@ -555,14 +556,13 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint32_t meta_all[kMmaWarps][SW];  // head mask | valid tokens << 8 of each slot's tile
   __shared__ int warp_tot[32];
-  __shared__ int s_asg[4];
+  __shared__ int s_asg[5];
   __shared__ int s_last, s_fail;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   uint32_t* meta = meta_all[w];
-  // shared memory: [rings | ring barriers | the CTA's result]
+  // shared memory: [rings | ring barriers]
   unsigned char* ring = smem + (size_t)w * SW * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)kMmaWarps * SW * stage_bytes) + w * SW;
-  float* part_s = reinterpret_cast<float*>(smem + (size_t)kMmaWarps * SW * (stage_bytes + 8));  // [G][kOut]
   if (lane == 0) {
     for (int s = 0; s < SW; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
@@ -575,8 +575,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
   const int bg = s_asg[0], split = s_asg[1], ns = s_asg[2], slot0 = s_asg[3];
   const int b = bg / p.Hkv, g = bg - b * p.Hkv;
   const uint32_t* list = p.lists + (size_t)bg * p.ustride;
-  const int U = min((int)__ldcg(list), p.umax);
-  const int tail_valid = (int)__ldcg(list + 1);
+  const int U = s_asg[4];  // list[0], as the compact count array holds it
   const int T = U * p.tpp;
   const int per = (T + ns - 1) / ns;
   const int lo = min(T, split * per), hi = min(T, lo + per);
@@ -597,7 +596,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
       const int t = lo + w + kMmaWarps * k;
       const int e = t / p.tpp, sub = t - e * p.tpp;
       const uint32_t en = __ldcg(list + 4 + e);
-      const int pv = (e == U - 1) ? tail_valid : p.page;
+      const int pv = (e == U - 1) ? (int)__ldcg(list + 1) : p.page;
       const uint32_t id = en & kNoPage;
       if (id != kNoPage && id >= (uint32_t)p.num_phys) set_err(p.err, BASISKV_DEVERR_BLOCK_TABLE);
       const int valid = (id < (uint32_t)p.num_phys) ? min(kTile, max(0, pv - sub * kTile)) : 0;
@@ -753,42 +752,51 @@ __global__ void __launch_bounds__(32 * kMmaWarps, kMmaCtasPerSm) attn_mma_kernel
     }
     __syncwarp();
   }
-  // the warps' states folded into part_s one warp after the other (a fixed
-  // order, so the result does not depend on timing)
+  // The warps' states, each [G][kOut] = (max, sum, o) per head, go to the
+  // first stage of the warp's own ring (free once its loop is done); then
+  // every thread combines the four warps' values of its elements in warp
+  // order (a fixed order, so the result does not depend on timing) into the
+  // CTA's slot.  After a timed-out wait a ring may still be receiving copies:
+  // it is not touched and the slot marks the heads' outputs NaN.
   l_run += __shfl_xor_sync(kFull, l_run, 1);
   l_run += __shfl_xor_sync(kFull, l_run, 2);
+  __syncthreads();  // s_fail is final
+  const bool failed = s_fail != 0;
+  if (!failed && head_ok) {
+    float* row = reinterpret_cast<float*>(ring) + gr * kOut;
+    if (tq == 0) {
+      row[0] = m_run;
+      row[1] = l_run;
+    }
+#pragma unroll
+    for (int jj = 0; jj < NT; ++jj) {
+      row[2 + 8 * jj + 2 * tq] = oacc[jj][0];
+      row[3 + 8 * jj + 2 * tq] = oacc[jj][1];
+    }
+  }
   __syncthreads();
-#pragma unroll 1
-  for (int ww = 0; ww < kMmaWarps; ++ww) {
-    if (w == ww) {
-      float* row = part_s + (size_t)gr * kOut;
-      float Mn = m_run, fs = 0.f, fw = 1.f;
-      if (head_ok) {
-        const float Ms = (ww == 0) ? -INFINITY : row[0];
-        Mn = fmaxf(Ms, m_run);
-        fs = (Ms == -INFINITY) ? 0.f : exp2f(Ms - Mn);
-        fw = (m_run == -INFINITY) ? 0.f : exp2f(m_run - Mn);
+  float* slot = p.part + (size_t)blockIdx.x * G * kOut;  // the group's CTAs, and slots, are consecutive
+  for (int i = threadIdx.x; i < G * kOut; i += blockDim.x) {
+    const int hh = i / kOut, col = i - hh * kOut;
+    float v = (col == 1) ? __int_as_float(0x7fc00000) : 0.f;  // a wait gave up: the head's output is NaN
+    if (!failed) {
+      float mw[kMmaWarps], M = -INFINITY;
 #pragma unroll
-        for (int jj = 0; jj < NT; ++jj)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float* a = row + 2 + 8 * jj + 2 * tq + e;
-            *a = (ww == 0 ? 0.f : *a * fs) + oacc[jj][e] * fw;
-          }
+      for (int ww = 0; ww < kMmaWarps; ++ww) {
+        mw[ww] = reinterpret_cast<const float*>(smem + (size_t)ww * SW * stage_bytes)[hh * kOut];
+        M = fmaxf(M, mw[ww]);
       }
-      __syncwarp();  // the row's four lanes have read row[0] before it changes
-      if (head_ok && tq == 0) {
-        row[1] = (ww == 0 ? 0.f : row[1] * fs) + l_run * fw;
-        row[0] = Mn;
+      if (col == 0) {
+        v = M;
+      } else {
+        v = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kMmaWarps; ++ww) {
+          const float s = (mw[ww] == -INFINITY) ? 0.f : exp2f(mw[ww] - M);
+          v = fmaf(reinterpret_cast<const float*>(smem + (size_t)ww * SW * stage_bytes)[i], s, v);
+        }
       }
     }
-    __syncthreads();
-  }
-  float* slot = p.part + (size_t)blockIdx.x * G * kOut;  // the group's CTAs, and slots, are consecutive
-  const bool failed = s_fail != 0;
-  for (int i = threadIdx.x; i < G * kOut; i += blockDim.x) {
-    float v = part_s[i];
-    if (failed && (i % kOut) == 1) v = __int_as_float(0x7fc00000);  // a wait gave up: the head's output is NaN
     slot[i] = v;
   }
   // the last CTA of the group to finish merges every split of its G heads
