@@ -532,6 +532,8 @@ def run_ours(args, world, rank, local):
         ra_gbs = (nbytes["route"] + nbytes["decode_attn"]) / ((mean["append_route"] + mean["decode_attn"]) * 1e-3) / 1e9
         # the committed counters are for per-head routing (other routings read other pages)
         traffic_rec = profiled_traffic("decode_attn.cu") if args.routing == "head" else None
+        if traffic_rec and (traffic_rec.get("workload") != full_wl.name or args.context):
+            traffic_rec = None  # the counters were taken on another workload
         roofline = {
             "kernel": "basiskv_decode_attn (one launch: union slice, attention, split merge)",
             "bound": "hbm", "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
@@ -562,7 +564,7 @@ def run_ours(args, world, rank, local):
                             exchange()
                             hy.copy_(eng.y, non_blocking=True)
                         else:
-                            eng.graph_step_host(hin, hy)   # copy in, step, copy out: one graph
+                            eng.graph_step_host(hin, hy)   # inputs in by a copy kernel, step, y stored on the host: one graph
                         if record:
                             b_.record(stream)
                             out.append((a, b_))
@@ -577,6 +579,7 @@ def run_ours(args, world, rank, local):
             e2e_ms = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in pairs), world, dev)
             e2e = {"value": round(tokens_per_step * args.steps / (e2e_ms / 1e3), 1), "unit": UNIT,
                    "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+                   "path": "copy-engine copies of pinned tensors" if args.tp else "basiskv_copy kernel in, out_proj stores y on the host",
                    "ms_per_step": round(e2e_ms / args.steps, 4)}
 
     prefill = None
