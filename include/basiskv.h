@@ -17,8 +17,10 @@
  *                        Value latents (rank-r output per head)
  *   basiskv_out_proj     (step 5)   y = sum_h o_h G_h through the fused factor
  *
- * A step whose inputs and output live in page-locked host memory brings the
- * inputs in with basiskv_copy and lets basiskv_out_proj store y on the host.
+ * basiskv_append_route does steps 1-3 in one call, the route's scoring running
+ * beside the append (no second stream needed).  A step whose inputs and output
+ * live in page-locked host memory brings the inputs in with basiskv_copy and
+ * lets basiskv_out_proj store y on the host.
  *
  * Method: "BasisKV: Value Latents for Communication and Key Routing"
  * (weekinpapers.com/paper/2611.02583v1, Abstract) and the kongchang.com
@@ -239,6 +241,26 @@ BASISKV_API basiskv_status basiskv_route_group(const basiskv_config* cfg, const 
                                    const void* q, int32_t batch, int32_t reduce, int32_t* sel,
                                    int32_t* sel_cnt, float* scores, void* workspace,
                                    size_t workspace_bytes, int32_t* err_flag, void* stream);
+
+/*
+ * Steps 1-3 of one decode step in one call: basiskv_append with n_new = 1
+ * (k_new, v_new as there), then basiskv_route (reduce = 0) or
+ * basiskv_route_group (reduce = BASISKV_GROUP_SUM / BASISKV_GROUP_MAX) with
+ * scores = NULL, on one stream.  Results are those of the two calls in that
+ * order.  The route's scoring kernel is launched as a programmatic dependent of
+ * the append kernel and runs beside it: without a scores output it reads no
+ * page the append writes (the recent page is kept whatever it scores), and it
+ * waits for the append before it completes, so everything after this call on
+ * the stream sees both.  Saves the second stream and the join a caller would
+ * otherwise use to overlap the two.  Arguments and errors as for the two calls
+ * (an invalid `reduce` returns BASISKV_ERR_INVALID_ARG); validation happens
+ * before either kernel is launched.
+ */
+BASISKV_API basiskv_status basiskv_append_route(const basiskv_config* cfg, const basiskv_cache* cache,
+                                                const basiskv_factors* factors, const void* k_new,
+                                                const void* v_new, const void* q, int32_t batch, int32_t reduce,
+                                                int32_t* sel, int32_t* sel_cnt, void* workspace,
+                                                size_t workspace_bytes, int32_t* err_flag, void* stream);
 
 /*
  * Step 4.  Exact sparse attention.  For each (b, h): over the valid tokens j

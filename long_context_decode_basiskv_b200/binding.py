@@ -27,7 +27,7 @@ SYMBOLS = [
     "basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
     "basiskv_fuse_out_factor", "basiskv_workspace_bytes", "basiskv_status_string",
     "basiskv_abi_version", "basiskv_decode_attn_noalloc", "basiskv_route_group", "basiskv_prefill",
-    "basiskv_copy",
+    "basiskv_copy", "basiskv_append_route",
 ]
 
 
@@ -72,6 +72,7 @@ def lib():
     L.basiskv_decode_attn_noalloc.argtypes = [pc, pk, vp, i32, vp, vp, vp, vp, vp]
     L.basiskv_fuse_out_factor.argtypes = [pc, vp, vp, vp, vp]
     L.basiskv_copy.argtypes = [vp, vp, sz, vp]
+    L.basiskv_append_route.argtypes = [pc, pk, pf, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp, vp]
     L.basiskv_workspace_bytes.argtypes = [pc, i32, i32]
     L.basiskv_workspace_bytes.restype = sz
     L.basiskv_status_string.argtypes = [i32]
@@ -79,7 +80,7 @@ def lib():
     L.basiskv_abi_version.argtypes = []
     for name in ["basiskv_append", "basiskv_route", "basiskv_decode_attn", "basiskv_out_proj",
                  "basiskv_fuse_out_factor", "basiskv_abi_version", "basiskv_decode_attn_noalloc",
-                 "basiskv_route_group", "basiskv_prefill", "basiskv_copy"]:
+                 "basiskv_route_group", "basiskv_prefill", "basiskv_copy", "basiskv_append_route"]:
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -252,6 +253,24 @@ def route(cfg: Config, cache: PagedCache, q: torch.Tensor, sel: torch.Tensor, se
     _check(lib().basiskv_route(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), _ptr(q), B, _ptr(sel),
                                _ptr(sel_cnt), _ptr(scores), _ptr(ws), ws.numel(), _ptr(err),
                                _stream(stream)), "basiskv_route")
+
+
+def append_route(cfg: Config, cache: PagedCache, f: Factors, k_new: torch.Tensor, v_new: torch.Tensor,
+                 q: torch.Tensor, reduce: int, sel: torch.Tensor, sel_cnt: torch.Tensor, ws: torch.Tensor,
+                 err: torch.Tensor, stream=None):
+    """append (one token per sequence) then route (reduce = 0) or route_group in one call,
+    the scoring running beside the append (basiskv_append_route)."""
+    B = q.shape[0]
+    _need(k_new, "k_new", cfg.dtype, (B, 1, cfg.num_kv_heads, cfg.head_dim))
+    _need(v_new, "v_new", cfg.dtype, (B, 1, cfg.num_kv_heads, cfg.head_dim))
+    _need(q, "q", cfg.dtype, (B, cfg.num_q_heads, cfg.head_dim))
+    _need(sel, "sel", torch.int32, (B, cfg.num_q_heads, cfg.top_k + 2))
+    _need(sel_cnt, "sel_cnt", torch.int32, (B, cfg.num_q_heads))
+    _need(ws, "workspace", torch.uint8)
+    _need(err, "err", torch.int32)
+    _check(lib().basiskv_append_route(ctypes.byref(cfg.c()), ctypes.byref(cache.c()), ctypes.byref(f.c()),
+                                      _ptr(k_new), _ptr(v_new), _ptr(q), B, reduce, _ptr(sel), _ptr(sel_cnt),
+                                      _ptr(ws), ws.numel(), _ptr(err), _stream(stream)), "basiskv_append_route")
 
 
 def route_group(cfg: Config, cache: PagedCache, q: torch.Tensor, reduce: int, sel: torch.Tensor,

@@ -201,7 +201,8 @@ basiskv_status basiskv_prefill(const basiskv_config* cfg, const basiskv_cache* c
 
 static basiskv_status route_common(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
                                    int32_t batch, int group_mode, int32_t* sel, int32_t* sel_cnt, float* scores,
-                                   void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
+                                   void* ws, size_t ws_bytes, int32_t* err_flag, void* stream,
+                                   const AppendParams* append_first = nullptr) {
   basiskv_status s = check_config(cfg);
   if (s != BASISKV_OK) return s;
   if ((s = check_cache(cfg, cache, false)) != BASISKV_OK) return s;
@@ -219,7 +220,13 @@ static basiskv_status route_common(const basiskv_config* cfg, const basiskv_cach
                  cache->num_phys_pages, cfg->top_k, scores ? 1 : 0, group_mode,
                  lists, reinterpret_cast<uint32_t*>(wsb + w.decode + w.plan.ucount_off),
                  reinterpret_cast<int32_t*>(wsb + w.rcnt), acnt, w.plan.ustride};
-  return cuda_status(launch_route(rp, cfg->head_dim, cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream));
+  if (append_first) {
+    // the append, then the scoring as its programmatic dependent (it reads none of the append's pages)
+    const cudaError_t e = launch_append(*append_first, cfg->dtype == BASISKV_BF16, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return cuda_status(launch_route(rp, cfg->head_dim, cfg->dtype == BASISKV_BF16, num_sms(), (cudaStream_t)stream,
+                                  append_first != nullptr));
 }
 
 basiskv_status basiskv_route(const basiskv_config* cfg, const basiskv_cache* cache, const void* q,
@@ -233,6 +240,24 @@ basiskv_status basiskv_route_group(const basiskv_config* cfg, const basiskv_cach
                                    float* scores, void* ws, size_t ws_bytes, int32_t* err_flag, void* stream) {
   if (reduce != BASISKV_GROUP_SUM && reduce != BASISKV_GROUP_MAX) return BASISKV_ERR_INVALID_ARG;
   return route_common(cfg, cache, q, batch, reduce, sel, sel_cnt, scores, ws, ws_bytes, err_flag, stream);
+}
+
+basiskv_status basiskv_append_route(const basiskv_config* cfg, const basiskv_cache* cache,
+                                    const basiskv_factors* f, const void* k_new, const void* v_new, const void* q,
+                                    int32_t batch, int32_t reduce, int32_t* sel, int32_t* sel_cnt, void* ws,
+                                    size_t ws_bytes, int32_t* err_flag, void* stream) {
+  basiskv_status s = check_config(cfg);
+  if (s != BASISKV_OK) return s;
+  if ((s = check_cache(cfg, cache, true)) != BASISKV_OK) return s;
+  if (reduce != 0 && reduce != BASISKV_GROUP_SUM && reduce != BASISKV_GROUP_MAX) return BASISKV_ERR_INVALID_ARG;
+  if (batch == 0) return BASISKV_OK;
+  if (!f || !f->A || !f->P || !f->E || !k_new || !v_new || !err_flag || batch < 0) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(f->A) || !aligned16(f->P) || !aligned16(f->E)) return BASISKV_ERR_INVALID_ARG;
+  const AppendParams ap{k_new, v_new, f->A, f->P, f->E, cache->k_raw, cache->c_lat, cache->r_res,
+                        cache->summary, cache->block_table, cache->seq_len, err_flag,
+                        batch, 1, cfg->num_kv_heads, cfg->head_dim, cfg->rank_v, cfg->rank_k,
+                        cfg->page_size, cache->max_pages, cache->num_phys_pages};
+  return route_common(cfg, cache, q, batch, reduce, sel, sel_cnt, nullptr, ws, ws_bytes, err_flag, stream, &ap);
 }
 
 basiskv_status basiskv_decode_attn(const basiskv_config* cfg, const basiskv_cache* cache,

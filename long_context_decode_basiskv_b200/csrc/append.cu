@@ -205,6 +205,10 @@ template <typename T>
 __global__ void __launch_bounds__(kDecThreads) append_decode_kernel(AppendParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int s_ok;
+  // A kernel launched as this one's programmatic dependent (the route's scoring
+  // in basiskv_append_route) may start now: it reads nothing this kernel writes
+  // and waits for it before it ends.
+  allow_dependents();
   const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int d = p.d, r = p.r, s = p.s, P = p.page;
   const int L = p.seq_len[b];

@@ -45,7 +45,10 @@ struct RouteParams {
   int32_t* acnt;    // [B][Hkv] the attention kernel's split counters, zeroed with the lists
   int ustride;
 };
-cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st);
+// beside_append: the score kernel is launched as a programmatic dependent of
+// the kernel before it, which must be the decode-step append (basiskv_append_route)
+cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st,
+                         bool beside_append = false);
 
 // Union lists from a given selection (sel / sel_cnt rows of every head).
 struct UnionParams {

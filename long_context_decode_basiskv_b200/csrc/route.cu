@@ -63,6 +63,15 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
   __shared__ __align__(16) float sq[G * D];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Launched as a programmatic dependent of the step's append (see
+  // launch_route), this kernel runs beside it: it reads no page the append
+  // writes, except with all_pages (the recent page's summary), when it waits
+  // for the append first.  The first CTA waits for the append before it ends,
+  // so the grid completes after the append and the kernels after it see the
+  // append's writes; the other CTAs leave as soon as they are done (a grid of
+  // more than one wave keeps its slots turning over).  In an ordinary launch
+  // both waits return at once.
+  if (p.all_pages) grid_dep_wait();
   // the length, this lane's block-table entry and the query rows are loaded
   // together (the entry is validated once the length is known)
   const int pw0 = c * kScoreCtaPages + warp * kScoreWarpPages;
@@ -74,7 +83,7 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
     if (c == 0 && tid == 0) set_err(p.err, BASISKV_DEVERR_SEQ_LEN);
     n = p.max_pages;
   }
-  if (c * kScoreCtaPages >= n) return;  // the whole CTA is past the last page
+  if (c * kScoreCtaPages >= n) return;  // the whole CTA is past the last page (never the first CTA)
   const size_t qrow = (size_t)b * p.Hq + (size_t)g * G;
   const T* qb = static_cast<const T*>(p.q) + qrow * D;
   for (int i = tid; i < G * D; i += kScoreThreads) sq[i] = Elem<T>::to_f(qb[i]);
@@ -168,6 +177,7 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
       }
     }
   }
+  if (c == 0 && g == 0 && b == 0) grid_dep_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -657,27 +667,35 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_hist_kernel(Route
 // launch
 // ---------------------------------------------------------------------------
 template <typename T, int D>
-static cudaError_t launch_score_g(const RouteParams& p, int G, cudaStream_t st) {
+static cudaError_t launch_score_g(const RouteParams& p, int G, bool beside_append, cudaStream_t st) {
   const int nchunk = (p.max_pages + kScoreCtaPages - 1) / kScoreCtaPages;
-  const dim3 grid(nchunk, p.Hkv, p.batch);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nchunk, p.Hkv, p.batch);
+  cfg.blockDim = dim3(kScoreThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start while the append runs
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = beside_append ? 1 : 0;
   switch (G) {
-    case 1: route_score_kernel<T, D, 1><<<grid, kScoreThreads, 0, st>>>(p); break;
-    case 2: route_score_kernel<T, D, 2><<<grid, kScoreThreads, 0, st>>>(p); break;
-    case 4: route_score_kernel<T, D, 4><<<grid, kScoreThreads, 0, st>>>(p); break;
-    case 8: route_score_kernel<T, D, 8><<<grid, kScoreThreads, 0, st>>>(p); break;
+    case 1: return cudaLaunchKernelEx(&cfg, route_score_kernel<T, D, 1>, p);
+    case 2: return cudaLaunchKernelEx(&cfg, route_score_kernel<T, D, 2>, p);
+    case 4: return cudaLaunchKernelEx(&cfg, route_score_kernel<T, D, 4>, p);
+    case 8: return cudaLaunchKernelEx(&cfg, route_score_kernel<T, D, 8>, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
-cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st) {
+cudaError_t launch_route(const RouteParams& p, int d, bool bf16, int num_sms, cudaStream_t st, bool beside_append) {
   (void)num_sms;
   const int G = p.Hq / p.Hkv;
   cudaError_t e;
+  const bool pa = beside_append;
   if (bf16)
-    e = (d == 128) ? launch_score_g<__nv_bfloat16, 128>(p, G, st) : launch_score_g<__nv_bfloat16, 64>(p, G, st);
+    e = (d == 128) ? launch_score_g<__nv_bfloat16, 128>(p, G, pa, st) : launch_score_g<__nv_bfloat16, 64>(p, G, pa, st);
   else
-    e = (d == 128) ? launch_score_g<float, 128>(p, G, st) : launch_score_g<float, 64>(p, G, st);
+    e = (d == 128) ? launch_score_g<float, 128>(p, G, pa, st) : launch_score_g<float, 64>(p, G, pa, st);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.group_mode ? p.Hkv : p.Hq, p.batch);
   if (p.max_pages <= kSelectThreads * 32) {

@@ -3,12 +3,16 @@
 ``DecodeEngine`` owns the device state of a batch: the paged cache (built by
 the library's own append kernel in prefill mode), the factors with the fused
 out-projection factor (built by the library's fusion kernel), the step's
-inputs and outputs, and one workspace.  ``step()`` enqueues the four calls of
-one decode step: append, route, decode_attn, out_proj.  ``routing`` picks one
+inputs and outputs, and one workspace.  ``step()`` enqueues one decode step:
+append and route (one basiskv_append_route call, or the two calls on two
+streams), decode_attn, out_proj.  ``routing`` picks one
 selection per query head ("head") or per KV group from the sum ("group_sum")
 or maximum ("group_max") of its heads' page scores.  ``prefill_mode`` builds
 the cache with basiskv_append ("exact", fp64 sums) or basiskv_prefill ("tc",
-the tensor-core path for long appends).
+the tensor-core path for long appends).  ``overlap`` picks how append and
+route overlap: "pdl" (one call, basiskv_append_route: the scoring runs
+beside the append as its programmatic dependent, one stream) or "streams"
+(basiskv_append on a forked stream beside basiskv_route, then a join).
 """
 from __future__ import annotations
 
@@ -29,9 +33,12 @@ _GROUP_REDUCE = {"group_sum": bk.GROUP_SUM, "group_max": bk.GROUP_MAX}
 
 class DecodeEngine:
     def __init__(self, case: Case, device="cuda", stream=None, routing: str = "head",
-                 prefill_mode: str = "exact"):
+                 prefill_mode: str = "exact", overlap: str = "pdl"):
         if routing != "head" and routing not in _GROUP_REDUCE:
             raise ValueError(f"routing must be 'head', 'group_sum' or 'group_max', not {routing!r}")
+        if overlap not in ("pdl", "streams"):
+            raise ValueError(f"overlap must be 'pdl' or 'streams', not {overlap!r}")
+        self.overlap = overlap
         if prefill_mode not in ("exact", "tc"):
             raise ValueError(f"prefill_mode must be 'exact' or 'tc', not {prefill_mode!r}")
         self.routing = routing
@@ -115,28 +122,48 @@ class DecodeEngine:
         receives the result straight from the kernel."""
         bk.out_proj(self.cfg, self.factors, self.o_lat, self.y if y is None else y, self.ws, stream)
 
-    def append_route(self, stream=None):
+    def append_route(self, stream=None, host_in=None):
         """Append (on a forked stream) concurrently with route, then join.
 
         Without a scores output, route reads nothing the step's append writes
         (only the recent page changes, and it is kept whatever it scores).
+        With `host_in` (pinned, input_buffer()'s layout) the step's inputs are
+        first brought in by basiskv_copy: with overlap "pdl" all of them in one
+        copy before the combined call; with "streams" k_new and v_new on the
+        forked stream before the append and q on the calling stream before
+        route.  (Measured in the step graph, the single copy before the
+        combined call is the faster of the two on every workload but the
+        64-sequence ragged batch.)
         """
         main = torch.cuda.current_stream(self.device) if stream is None else stream
         if not hasattr(self, "_aux"):
             self._aux = torch.cuda.Stream(device=self.device)
             self._fork = torch.cuda.Event()
             self._join = torch.cuda.Event()
+        nq = self.q.numel()
+        if self.overlap == "pdl":
+            if host_in is not None:
+                bk.copy(self._inbuf, host_in, main)
+            bk.append_route(self.cfg, self.cache, self.factors, self.k_new, self.v_new, self.q,
+                            0 if self.routing == "head" else _GROUP_REDUCE[self.routing], self.sel,
+                            self.sel_cnt, self.ws, self.err, main)
+            return
         self._fork.record(main)
         self._aux.wait_event(self._fork)
+        if host_in is not None:
+            bk.copy(self._inbuf[nq:], host_in[nq:], self._aux)
         self.append(self._aux)
         self._join.record(self._aux)
+        if host_in is not None:
+            bk.copy(self._inbuf[:nq], host_in[:nq], main)
         self.route(stream=main)
         main.wait_event(self._join)
 
-    def step(self, stream=None, y=None):
+    def step(self, stream=None, y=None, host_in=None):
         """One decode step: (append || route) -> decode_attn -> out_proj (into y, by
-        default the engine's device tensor)."""
-        self.append_route(stream)
+        default the engine's device tensor; inputs from `host_in` when given, see
+        append_route)."""
+        self.append_route(stream, host_in)
         self.decode_attn(stream)
         self.out_proj(stream, y)
         return self.y if y is None else y
@@ -160,7 +187,8 @@ class DecodeEngine:
     def graph_step_host(self, host_in: torch.Tensor, host_y: torch.Tensor):
         """One decode step with host buffers, replayed from one CUDA graph: the step's
         inputs come from `host_in` (pinned, input_buffer()'s layout and dtype) through
-        basiskv_copy, then the four calls, the out-projection storing y straight into
+        basiskv_copy (see append_route), the step's calls, the out-projection storing y
+        straight into
         `host_y` (pinned, y's shape and dtype); no copy-engine transfer.  The graph is
         captured on the first call for these two buffers; the caller refills host_in before
         a call and reads host_y once the current stream is synchronised."""
@@ -179,8 +207,7 @@ class DecodeEngine:
             torch.cuda.current_stream(self.device).wait_stream(side)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=side):
-                bk.copy(self._inbuf, host_in)
-                self.step(y=host_y)
+                self.step(y=host_y, host_in=host_in)
             self._io_graph, self._io_key = g, key
         self._io_graph.replay()
         return host_y

@@ -197,6 +197,31 @@ def test_route_group_checks(L):
                                      1 << 30, 256, None) == bk.ERR_INVALID_ARG   # misaligned q
 
 
+def test_append_route_checks(L):
+    """basiskv_append_route: the append's and the route's checks, all before any launch
+    (reduce 0 = per head, else GROUP_SUM / GROUP_MAX)."""
+    cfg = _cfg()
+    good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
+    f = bk.CFactors(256, 256, 256, 256)
+
+    def call(cache=good, fac=f, k=256, v=256, q=256, batch=1, reduce=0, sel=256, ws=256, ws_bytes=1 << 30, err=256):
+        return L.basiskv_append_route(ctypes.byref(cfg), ctypes.byref(cache) if cache else None,
+                                      ctypes.byref(fac) if fac else None, k, v, q, batch, reduce, sel, 256, ws,
+                                      ws_bytes, err, None)
+
+    for bad in (3, -1, 7):
+        assert call(reduce=bad) == bk.ERR_INVALID_ARG
+    assert call(batch=0) == bk.OK                                  # nothing to do
+    assert call(cache=None) == bk.ERR_INVALID_ARG
+    assert call(fac=None) == bk.ERR_INVALID_ARG
+    assert call(k=None) == bk.ERR_INVALID_ARG
+    assert call(err=None) == bk.ERR_INVALID_ARG
+    assert call(q=260) == bk.ERR_INVALID_ARG                       # misaligned q
+    assert call(ws=None) == bk.ERR_WORKSPACE
+    assert call(ws_bytes=64) == bk.ERR_WORKSPACE
+    assert call(fac=bk.CFactors(260, 256, 256, 256)) == bk.ERR_INVALID_ARG   # misaligned A
+
+
 def test_prefill_checks(L):
     """basiskv_prefill: bf16 with ranks that are multiples of 16 only; otherwise basiskv_append's checks."""
     good = bk.CCache(256, 256, 256, 256, 256, 256, 10, 10)
