@@ -349,19 +349,24 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
 // page summaries of every page the appended tokens touched
 // ---------------------------------------------------------------------------
 // One CTA per (sequence, KV head, run of kSumTokens / page pages).  All of the
-// run's stored C and R blocks (contiguous per page) come into shared memory in
-// one round of 16-byte cp.async copies, then: the column means of each page's
-// valid tokens in fp64 (tokens in order), and S[x] = sum_j mean(C)_j P[j][x] +
-// sum_q mean(R)_q E[x][q] in fp64, rounded once.  E is staged transposed so
-// that consecutive x read consecutive words.
+// run's stored C and R blocks (contiguous per page) and the head's P factor
+// (bf16) come into shared memory in one round of 16-byte cp.async copies.
+// Then the column means of each page's valid tokens in fp64 (tokens in
+// order; one thread per column, the run's pages interleaved), and S[x] =
+// sum_j mean(C)_j P[j][x] + sum_q mean(R)_q E[x][q] in fp64, rounded once:
+// one thread per x with the run's pages as independent chains, P[j][x] read
+// once for all of them, row x of E read from global memory 8 elements at a
+// time.  Per output the sums run in the same order as before the pages were
+// interleaved, so the values are unchanged.
 constexpr int kSumTokens = 128;  // tokens (pages x page size) per CTA
 constexpr int kSumThreads = 128;
+constexpr int kSumMaxPages = kSumTokens / 16;  // pages per CTA at the smallest page size
 
 static int sum_pages(int page) { return std::max(1, kSumTokens / page); }
 static size_t sum_smem_bytes(int d, int r, int s, int page) {
   const int np = sum_pages(page);
-  return (size_t)(r * d + d * s) * sizeof(float) + (size_t)np * page * (r + s) * 2 +
-         (size_t)np * (r + s) * sizeof(double) + 16 * sizeof(int);
+  return (size_t)r * d * 2 + (size_t)np * page * (r + s) * 2 + (size_t)(r + s) * kSumMaxPages * sizeof(double) +
+         16 * sizeof(int);
 }
 
 __global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams p, int np) {
@@ -375,18 +380,17 @@ __global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams 
   const int pg0 = first_page + blockIdx.x * np;
   if (pg0 > last_page) return;
   const int npg = min(np, last_page - pg0 + 1);  // pages of this CTA
-  float* sP = reinterpret_cast<float*>(smem);                          // [r][d]
-  float* sEt = sP + r * d;                                             // [s][d] (E transposed)
-  __nv_bfloat16* sCR = reinterpret_cast<__nv_bfloat16*>(sEt + d * s);  // per page: C [P][r], R [P][s]
-  double* sMean = reinterpret_cast<double*>(sCR + (size_t)np * P * (r + s));  // [np][r + s]
-  int* sPhys = reinterpret_cast<int*>(sMean + (size_t)np * (r + s));          // [np]
+  __nv_bfloat16* sP = reinterpret_cast<__nv_bfloat16*>(smem);          // [r][d]
+  __nv_bfloat16* sCR = sP + (size_t)r * d;                            // per page: C [P][r], R [P][s]
+  double* sMean = reinterpret_cast<double*>(sCR + (size_t)np * P * (r + s));  // [r + s][kSumMaxPages]
+  int* sPhys = reinterpret_cast<int*>(sMean + (size_t)(r + s) * kSumMaxPages);  // [np]
   const size_t blk_elems = (size_t)P * (r + s);
   if (tid < npg) {
     const int ph = p.block_table[(size_t)b * p.max_pages + pg0 + tid];
     sPhys[tid] = (ph < 0 || ph >= p.num_phys) ? -1 : ph;  // reported by the latent kernel
   }
   __syncthreads();
-  // this run's C and R blocks, every copy in flight at once
+  // this run's C and R blocks and the factor P, every copy in flight at once
   const int c_pieces = P * r * 2 / 16, r_pieces = P * s * 2 / 16;
   const __nv_bfloat16* clat = static_cast<const __nv_bfloat16*>(p.c_lat);
   const __nv_bfloat16* rres = static_cast<const __nv_bfloat16*>(p.r_res);
@@ -401,45 +405,70 @@ __global__ void __launch_bounds__(kSumThreads) page_summary_kernel(AppendParams 
     else
       cp_async16_cg(dst + (size_t)P * r + (x - c_pieces) * 8, rres + blk * P * s + (x - c_pieces) * 8);
   }
-  cp_async_commit_group();
-  // the factors meanwhile (fp32, E transposed)
   const __nv_bfloat16* Pm = static_cast<const __nv_bfloat16*>(p.P) + (size_t)g * r * d;
-  const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(p.E) + (size_t)g * d * s;
-  for (int i = tid; i < r * d; i += kSumThreads) sP[i] = __bfloat162float(Pm[i]);
-  for (int i = tid; i < d * s; i += kSumThreads) {
-    const int x = i / s, q = i - x * s;
-    sEt[q * d + x] = __bfloat162float(E[i]);
-  }
+  for (int i = tid; i < r * d / 8; i += kSumThreads) cp_async16_cg(sP + i * 8, Pm + i * 8);
+  cp_async_commit_group();
   cp_async_wait_group<0>();
   __syncthreads();
   // column means of every page's valid tokens (fp64, tokens in order)
   const bool swz_on = kc_swizzled(true, d, r);
   const int mc = swz_on ? swz_mask(r) : 0;
-  for (int i = tid; i < npg * (r + s); i += kSumThreads) {
-    const int pi = i / (r + s), j = i - pi * (r + s);
-    if (sPhys[pi] < 0) continue;
+  int m[kSumMaxPages];
+#pragma unroll
+  for (int pi = 0; pi < kSumMaxPages; ++pi) {
     const int page = pg0 + pi;
-    const int m = min(L, (page + 1) * P) - page * P;
-    const __nv_bfloat16* blkp = sCR + (size_t)pi * blk_elems;
-    double acc = 0.0;
-    if (j < r) {
-      for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(blkp[t * r + swz(j, t, mc)]);
-    } else {
-      for (int t = 0; t < m; ++t) acc += (double)__bfloat162float(blkp[(size_t)P * r + t * s + (j - r)]);
+    m[pi] = (pi < npg) ? min(L, (page + 1) * P) - page * P : 0;
+  }
+  for (int j = tid; j < r + s; j += kSumThreads) {
+    double acc[kSumMaxPages];
+#pragma unroll
+    for (int pi = 0; pi < kSumMaxPages; ++pi) acc[pi] = 0.0;
+    for (int t = 0; t < P; ++t) {
+#pragma unroll
+      for (int pi = 0; pi < kSumMaxPages; ++pi) {
+        if (t < m[pi]) {
+          const __nv_bfloat16* blkp = sCR + (size_t)pi * blk_elems;
+          const __nv_bfloat16 v = (j < r) ? blkp[t * r + swz(j, t, mc)] : blkp[(size_t)P * r + t * s + (j - r)];
+          acc[pi] += (double)__bfloat162float(v);
+        }
+      }
     }
-    sMean[(size_t)pi * (r + s) + j] = acc / (double)m;
+#pragma unroll
+    for (int pi = 0; pi < kSumMaxPages; ++pi)
+      if (m[pi] > 0) sMean[(size_t)j * kSumMaxPages + pi] = acc[pi] / (double)m[pi];
   }
   __syncthreads();
-  for (int i = tid; i < npg * d; i += kSumThreads) {
-    const int pi = i / d, x = i - pi * d;
-    if (sPhys[pi] < 0) continue;
-    const double* mean = sMean + (size_t)pi * (r + s);
-    double acc = 0.0;
-    for (int j = 0; j < r; ++j) acc = fma(mean[j], (double)sP[j * d + x], acc);
-    double acc2 = 0.0;
-    for (int q = 0; q < s; ++q) acc2 = fma(mean[r + q], (double)sEt[q * d + x], acc2);
-    const size_t blk = (size_t)sPhys[pi] * p.Hkv + g;
-    p.summary[blk * d + x] = __double2float_rn(acc + acc2);
+  const __nv_bfloat16* E = static_cast<const __nv_bfloat16*>(p.E) + (size_t)g * d * s;
+  for (int x = tid; x < d; x += kSumThreads) {
+    double acc[kSumMaxPages], acc2[kSumMaxPages];
+#pragma unroll
+    for (int pi = 0; pi < kSumMaxPages; ++pi) acc[pi] = acc2[pi] = 0.0;
+    for (int j = 0; j < r; ++j) {
+      const double pj = (double)__bfloat162float(sP[j * d + x]);
+      const double* mj = sMean + (size_t)j * kSumMaxPages;
+#pragma unroll
+      for (int pi = 0; pi < kSumMaxPages; ++pi)
+        if (pi < npg) acc[pi] = fma(mj[pi], pj, acc[pi]);
+    }
+    const uint4* erow = reinterpret_cast<const uint4*>(E + (size_t)x * s);  // row x of E, 8 elements a load
+    for (int q0 = 0; q0 < s; q0 += 8) {
+      const uint4 w = __ldg(erow + q0 / 8);
+      const __nv_bfloat16* e8 = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const double eq = (double)__bfloat162float(e8[u]);
+        const double* mq = sMean + (size_t)(r + q0 + u) * kSumMaxPages;
+#pragma unroll
+        for (int pi = 0; pi < kSumMaxPages; ++pi)
+          if (pi < npg) acc2[pi] = fma(mq[pi], eq, acc2[pi]);
+      }
+    }
+#pragma unroll
+    for (int pi = 0; pi < kSumMaxPages; ++pi) {
+      if (pi >= npg || sPhys[pi] < 0) continue;
+      const size_t blk = (size_t)sPhys[pi] * p.Hkv + g;
+      p.summary[blk * d + x] = __double2float_rn(acc[pi] + acc2[pi]);
+    }
   }
 }
 
