@@ -72,12 +72,12 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
 }
 
 struct PfLayout {
-  uint32_t b1, b2, b3, v, k, chi, clo, bar, slot, total;
+  uint32_t b1, b2, b3, v, k, v2, k2, chi, clo, bar, slot, total;
 };
 
 __host__ __device__ inline int pf_atoms(int kdim) { return (kdim + 63) / 64; }
 
-__host__ __device__ inline PfLayout pf_layout(int d, int r, int s) {
+__host__ __device__ inline PfLayout pf_layout(int d, int r, int s, bool two_tiles = true) {
   PfLayout L{};
   uint32_t o = 0;
   L.b1 = o;  o += (uint32_t)pf_atoms(d) * r * 128;  // A_g^T: r rows, K = d
@@ -85,12 +85,23 @@ __host__ __device__ inline PfLayout pf_layout(int d, int r, int s) {
   L.b3 = o;  o += (uint32_t)pf_atoms(d) * s * 128;  // E_g^T: s rows, K = d
   L.v = o;   o += (uint32_t)pf_atoms(d) * kAtom;    // V tile, then (K - X) hi
   L.k = o;   o += (uint32_t)pf_atoms(d) * kAtom;    // K tile, then (K - X) lo
+  L.v2 = L.v;
+  L.k2 = L.k;
+  if (two_tiles) {  // the next tile's V and K, loading meanwhile
+    L.v2 = o;  o += (uint32_t)pf_atoms(d) * kAtom;
+    L.k2 = o;  o += (uint32_t)pf_atoms(d) * kAtom;
+  }
   L.chi = o; o += (uint32_t)pf_atoms(r) * kAtom;    // C hi
   L.clo = o; o += (uint32_t)pf_atoms(r) * kAtom;    // C lo
   L.bar = o; o += 16;
   L.slot = o; o += 16;
   L.total = o;
   return L;
+}
+// the double-buffered layout where it fits the shared memory, else one tile buffer
+__host__ __device__ inline PfLayout pf_layout_fit(int d, int r, int s) {
+  const PfLayout two = pf_layout(d, r, s, true);
+  return (two.total + 1024 <= 227 * 1024) ? two : pf_layout(d, r, s, false);
 }
 
 __host__ __device__ inline uint32_t pf_tmem_cols(int d, int r, int s) {
@@ -116,12 +127,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
   const int ntiles = (p.n_new + kPfM - 1) / kPfM;
   if ((int)blockIdx.x >= ntiles) return;
 
-  const PfLayout lay = pf_layout(d, r, s);
+  const PfLayout lay = pf_layout_fit(d, r, s);
+  const bool two_tiles = lay.v2 != lay.v;
   unsigned char* sB1 = smem + lay.b1;
   unsigned char* sB2 = smem + lay.b2;
   unsigned char* sB3 = smem + lay.b3;
-  unsigned char* sV = smem + lay.v;
-  unsigned char* sK = smem + lay.k;
+  // tile buffer i: V and K rows (i = 1 is buffer 0 again without room for two)
+  auto vbuf = [&](int i) { return smem + (i ? lay.v2 : lay.v); };
+  auto kbuf = [&](int i) { return smem + (i ? lay.k2 : lay.k); };
   unsigned char* sChi = smem + lay.chi;
   unsigned char* sClo = smem + lay.clo;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + lay.bar);
@@ -205,32 +218,36 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
     if (s_fail) ok = false;
   };
 
-  for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+  // k and v rows of tile `t` -> swizzled operand tiles of buffer `buf` by cp.async
+  // (zeros past the last token); one commit group per tile
+  auto load_tile = [&](int t, int buf) {
+    const int t0 = t * kPfM;
+    for (int q = tid; q < kPfM * cpr; q += kPfThreads) {
+      const int row = q / cpr, c = q - row * cpr;
+      const int tok = t0 + row;
+      const bool valid = tok < p.n_new;
+      const size_t src = valid ? (((size_t)b * p.n_new + tok) * p.Hkv + g) * d + (size_t)c * 8 : 0;
+      const uint32_t off = sw_off(row, c * 8, kPfM);
+      cp_async16_zfill(vbuf(buf) + off, vin + src, valid);
+      cp_async16_zfill(kbuf(buf) + off, kin + src, valid);
+    }
+    cp_async_commit_group();
+  };
+  load_tile(blockIdx.x, 0);
+  int it = 0;
+  for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
     const int t0 = tile * kPfM;
-    // k and v rows of the tile -> swizzled operand tiles, 8 chunks of each in flight per thread
-    for (int i0 = 0; i0 < kPfM * cpr / kPfThreads; i0 += 8) {
-      uint4 kq[8], vq[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int q = tid + kPfThreads * (i0 + u);
-        const int row = q / cpr, c = q - row * cpr;
-        const int tok = t0 + row;
-        kq[u] = make_uint4(0u, 0u, 0u, 0u);
-        vq[u] = kq[u];
-        if (tok < p.n_new) {
-          const size_t src = (((size_t)b * p.n_new + tok) * p.Hkv + g) * d + (size_t)c * 8;
-          kq[u] = __ldg(reinterpret_cast<const uint4*>(kin + src));
-          vq[u] = __ldg(reinterpret_cast<const uint4*>(vin + src));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int q = tid + kPfThreads * (i0 + u);
-        const int row = q / cpr, c = q - row * cpr;
-        const uint32_t off = sw_off(row, c * 8, kPfM);
-        *reinterpret_cast<uint4*>(sV + off) = vq[u];
-        *reinterpret_cast<uint4*>(sK + off) = kq[u];
-      }
+    unsigned char* const sV = vbuf(it & 1);
+    unsigned char* const sK = kbuf(it & 1);
+    if (two_tiles) {
+      // the next tile's rows load while this one is worked on (its buffer was the previous
+      // tile's, free since that tile's last barrier); then wait for this tile's rows
+      if (tile + (int)gridDim.x < ntiles) load_tile(tile + gridDim.x, (it + 1) & 1);
+      else cp_async_commit_group();
+      cp_async_wait_group<1>();
+    } else {
+      if (it > 0) load_tile(tile, 0);
+      cp_async_wait_group<0>();
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -336,6 +353,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(AppendParams 
     __syncthreads();  // smem tiles and TMEM are reused by the next tile
     tc_fence_after();
   }
+  cp_async_wait_group<0>();  // no copy may still be landing in shared memory when the CTA ends
   if (!ok && tid == 0) set_err(p.err, BASISKV_DEVERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
@@ -476,12 +494,12 @@ bool prefill_tc_supported(bool bf16, int d, int r, int s) {
   // head_dim 128 only: the shapes the parity tests exercise (64 would take the same code with one
   // K atom per operand, and is left to basiskv_append until it is tested)
   return bf16 && d == 128 && r >= 16 && r <= 128 && r % 16 == 0 && s >= 16 && s <= 64 &&
-         s % 16 == 0 && pf_layout(d, r, s).total + 1024 <= 227 * 1024 &&
+         s % 16 == 0 && pf_layout(d, r, s, false).total + 1024 <= 227 * 1024 &&
          sum_smem_bytes(d, r, s, 16) <= 227 * 1024;
 }
 
 cudaError_t launch_prefill_tc(const AppendParams& p, int num_sms, cudaStream_t st) {
-  const PfLayout lay = pf_layout(p.d, p.r, p.s);
+  const PfLayout lay = pf_layout_fit(p.d, p.r, p.s);
   const size_t smem = lay.total + 1024;  // + alignment of the dynamic window to 1024 bytes
   cudaError_t e = ensure_smem((const void*)prefill_tc_kernel, smem);
   if (e != cudaSuccess) return e;
