@@ -253,8 +253,8 @@ __device__ __forceinline__ uint32_t order_key(float v) {
 
 // Thread-block cluster helpers: this CTA's rank in its cluster; the cluster
 // barrier split into arrive (release) and wait (acquire), executed by every
-// thread of every CTA of the cluster; an OR into another CTA's shared memory
-// (the word at the address `local` has in this CTA, in CTA `rank`).
+// thread of every CTA of the cluster; a load from another CTA's shared memory
+// (ld_shared_cluster, below).
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
