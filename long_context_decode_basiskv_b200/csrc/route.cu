@@ -61,6 +61,9 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
   constexpr int DPL = D / 32;
   constexpr int N = kPagesPerWarp * G;
   __shared__ __align__(16) float sq[G * D];
+  // D = 128: each warp's next item of summary rows lands here (cp.async) while
+  // the current item is scored; lane l's 16 bytes of page i at [warp][i][l]
+  __shared__ __align__(16) float4 s_next[(DPL == 4) ? kScoreWarps : 1][kPagesPerWarp][32];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // Launched as a programmatic dependent of the step's append (see
@@ -104,13 +107,33 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
     for (int u = 0; u < DPL; ++u) qf[hi][u] = sq[hi * D + lane * DPL + u];
   float* outb = p.scores + qrow * p.max_pages;
   float* outg = p.scores + ((size_t)b * p.Hkv + g) * p.max_pages;  // the group's row (group modes)
+  // item i0's rows into this warp's s_next slot (zeros for a page not scored)
+  auto issue_next = [&](int i0) {
+#pragma unroll
+    for (int i = 0; i < kPagesPerWarp; ++i) {
+      const int ph = __shfl_sync(kFull, my_phys, i0 + i);
+      const float* rowp = (ph >= 0) ? p.summary + ((size_t)ph * p.Hkv + g) * D + lane * DPL : p.summary;
+      cp_async16_zfill(&s_next[(DPL == 4) ? warp : 0][i][lane], rowp, ph >= 0);
+    }
+    cp_async_commit_group();
+  };
 #pragma unroll 1
   for (int i0 = 0; i0 < kScoreWarpPages; i0 += kPagesPerWarp) {
     const int p0 = pw0 + i0;
     if (p0 >= n) break;
+    const bool staged = DPL == 4 && i0 > 0;  // this item was prefetched into s_next
     float sv[kPagesPerWarp][DPL];
+    if (staged) {
+      cp_async_wait_group<0>();
 #pragma unroll
-    for (int i = 0; i < kPagesPerWarp; ++i) {
+      for (int i = 0; i < kPagesPerWarp; ++i) {
+        const float4 v = s_next[(DPL == 4) ? warp : 0][i][lane];
+        sv[i][0] = v.x; sv[i][1] = v.y;
+        if constexpr (DPL == 4) { sv[i][2] = v.z; sv[i][3] = v.w; }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPagesPerWarp && !staged; ++i) {
       const int ph = __shfl_sync(kFull, my_phys, i0 + i);
       if (ph >= 0) {
         const float* rowp = p.summary + ((size_t)ph * p.Hkv + g) * D + lane * DPL;
@@ -136,6 +159,9 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
         for (int u = 0; u < DPL; ++u) a = fmaf(qf[hi][u], sv[i][u], a);
         part[i * G + hi] = a;
       }
+    // the next item's rows start coming in now: the reads of the slot above fed the
+    // products just issued, so they are done before the slot is written again
+    if (DPL == 4 && i0 + kPagesPerWarp < kScoreWarpPages && p0 + kPagesPerWarp < n) issue_next(i0 + kPagesPerWarp);
     transpose_reduce<N>(part, lane);
     float* out = outb + p0;
     if (p.group_mode != 0) {
@@ -177,6 +203,7 @@ __global__ void __launch_bounds__(kScoreThreads, (G >= 8) ? 2 : 4) route_score_k
       }
     }
   }
+  cp_async_wait_group<0>();  // no copy still landing in shared memory when the CTA ends
   if (c == 0 && g == 0 && b == 0) grid_dep_wait();
 }
 
