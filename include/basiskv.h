@@ -159,7 +159,10 @@ typedef struct {
  * the raw key is stored as given.  Then every touched page's summary is
  * recomputed over its valid tokens: S = mean(C) P_g + mean(R) E_g^T, rounded
  * to fp32.  n_new = 1 is the decode step; larger n_new is prefill.
- * factors->Gt is not read (it may be NULL).
+ * factors->Gt is not read (it may be NULL).  With n_new = 1 the kernel lets a
+ * programmatic dependent launch at its start: a kernel launched after this
+ * call with programmatic stream serialization must execute griddepcontrol.wait
+ * before it reads anything the append writes (ordinary launches are unaffected).
  * err_flag (device int32) may not be NULL.
  */
 BASISKV_API basiskv_status basiskv_append(const basiskv_config* cfg, const basiskv_cache* cache,
