@@ -51,13 +51,23 @@ def test_copy_refusals():
     torch.cuda.synchronize()
 
 
-def _engine(batch=3, name="host_io"):
-    wl = shrink(WORKLOADS["llama3_8b_32k"], batch=batch, context=16 * 200 + 5, top_k=24, name=name)
+# the three out-projection kernels: mma.sync (bf16, batch <= 8), tcgen05 (a K too
+# large for the mma kernel's shared memory), the fp32 one
+SHAPES = [
+    ("llama3_8b_32k", dict(batch=3, context=16 * 200 + 5, top_k=24)),
+    ("llama3_70b_64k", dict(batch=2, context=16 * 150 + 9, top_k=20)),
+    ("tiny_fp32", dict(batch=2, context=600, top_k=6)),
+]
+
+
+def _engine(base="llama3_8b_32k", kw=SHAPES[0][1], name="host_io"):
+    wl = shrink(WORKLOADS[base], name=name, **kw)
     return DecodeEngine(make_case(wl, "cuda"))
 
 
-def test_out_proj_into_pinned_host():
-    eng = _engine()
+@pytest.mark.parametrize("base,kw", SHAPES, ids=[s[0] for s in SHAPES])
+def test_out_proj_into_pinned_host(base, kw):
+    eng = _engine(base, kw)
     eng.step()
     torch.cuda.synchronize()
     hy = torch.full(tuple(eng.y.shape), float("nan"), dtype=torch.float32).pin_memory()
@@ -76,10 +86,13 @@ def test_out_proj_into_pinned_host():
     assert not np.any(pageable)
 
 
-def test_graph_step_host_matches_device_step():
+@pytest.mark.parametrize("overlap", ["pdl", "streams"])
+@pytest.mark.parametrize("base,kw", SHAPES, ids=[s[0] for s in SHAPES])
+def test_graph_step_host_matches_device_step(base, kw, overlap):
     """The host-buffer graph step (inputs in by basiskv_copy, y stored on the host) gives
     exactly the device step's y, for the captured inputs and for new ones."""
-    eng = _engine()
+    wl = shrink(WORKLOADS[base], name="host_io", **kw)
+    eng = DecodeEngine(make_case(wl, "cuda"), overlap=overlap)
     hin = eng.input_buffer().cpu().pin_memory()
     hy = torch.zeros(tuple(eng.y.shape), dtype=torch.float32).pin_memory()
     eng.graph_step()
