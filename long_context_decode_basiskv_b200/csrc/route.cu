@@ -297,10 +297,26 @@ __device__ __forceinline__ uint32_t select_rows_reg(const RouteParams& p, const 
   const float* sc = p.scores + rows.in * p.max_pages;
   const int p0 = tid * KPT;
   uint32_t key[KPT];
+  if ((p.max_pages & 3) == 0) {
+    // 16-byte rows: the thread's scores four at a time (every load inside the row:
+    // p0 + j + 4 <= n <= max_pages whenever p0 + j < n)
 #pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    const int pg = p0 + j;
-    key[j] = (pg >= 1 && pg <= n - 2) ? order_key(sc[pg]) : 0u;  // 0: not a candidate
+    for (int j = 0; j < KPT; j += 4) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (p0 + j < n) v = *reinterpret_cast<const float4*>(sc + p0 + j);
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int pg = p0 + j + u;
+        key[j + u] = (pg >= 1 && pg <= n - 2) ? order_key(vv[u]) : 0u;  // 0: not a candidate
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int pg = p0 + j;
+      key[j] = (pg >= 1 && pg <= n - 2) ? order_key(sc[pg]) : 0u;  // 0: not a candidate
+    }
   }
   auto count_ge = [&](uint32_t t) {
     int c = 0;
