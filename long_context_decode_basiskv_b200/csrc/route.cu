@@ -285,12 +285,12 @@ __device__ __forceinline__ void select_union_tail(const RouteParams& p, int b, i
                        (size_t)p.batch * p.Hkv, p.err, masks, bt_smem, warp_tot);
 }
 
-// The selection proper of route_select_kernel (n > top_k + 2 pages): writes
-// the CTA's sel rows and returns this thread's kept pages as bits (bit j:
-// page tid KPT + j).
+// The selection proper of route_select_kernel (n > top_k + 2 pages): returns
+// this thread's kept pages as bits (bit j: page tid KPT + j), the sel row
+// position of its first one and the row's count (put_kept writes them).
 template <int KPT>
 __device__ __forceinline__ uint32_t select_rows_reg(const RouteParams& p, const SelRows& rows, int n, int* red,
-                                                    int* warp_tot) {
+                                                    int* warp_tot, int& first_pos, int& total) {
   const int tid = threadIdx.x;
   const int kk = p.top_k;
   // thread t holds pages [t * KPT, t * KPT + KPT)
@@ -365,15 +365,25 @@ __device__ __forceinline__ uint32_t select_rows_reg(const RouteParams& p, const 
     const int pg = p0 + j;
     bool take = (pg == 0 || pg == n - 1 || key[j] > Tk) && pg < n;
     if (key[j] != 0u && key[j] == Tk) take = tie++ < keep_eq;
-    if (take) {
-      put_sel(p, rows, pos++, pg);
-      bits |= 1u << j;
-    }
+    if (take) bits |= 1u << j;
   }
-  const int total = above_tot + min(equal_tot, keep_eq);
-  for (int i = total + tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, -1);
-  if (tid == 0) put_cnt(p, rows, total);
+  first_pos = pos;
+  total = above_tot + min(equal_tot, keep_eq);
   return bits;
+}
+
+// The sel row entries of this thread's kept pages (bits from select_rows_reg,
+// positions from first_pos on), the row's unused tail (-1) and its count.
+template <int KPT>
+__device__ __forceinline__ void put_kept(const RouteParams& p, const SelRows& rows, uint32_t bits, int first_pos,
+                                         int total) {
+  const int tid = threadIdx.x, p0 = tid * KPT;
+  int pos = first_pos;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if ((bits >> j) & 1u) put_sel(p, rows, pos++, p0 + j);
+  for (int i = total + tid; i < p.top_k + 2; i += kSelectThreads) put_sel(p, rows, i, -1);
+  if (tid == 0) put_cnt(p, rows, total);
 }
 
 // One CTA per (sequence, query head), or per (sequence, KV group) in the group
@@ -410,16 +420,21 @@ __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParam
     cp_async_commit_group();
   }
   uint32_t take;
-  if (n <= kk + 2) {
+  int first_pos = 0, total = 0;
+  const bool ranked = n > kk + 2;
+  if (!ranked) {
     for (int i = tid; i < kk + 2; i += kSelectThreads) put_sel(p, rows, i, (i < n) ? i : -1);
     if (tid == 0) put_cnt(p, rows, n);
     const int m = min(KPT, max(0, n - p0));  // every page is kept
     take = (m >= 32) ? 0xffffffffu : ((1u << m) - 1u);
   } else {
-    take = select_rows_reg<KPT>(p, rows, n, red, warp_tot);
+    take = select_rows_reg<KPT>(p, rows, n, red, warp_tot, first_pos, total);
   }
   s_take[tid] = take;
   cluster_arrive_release();  // this CTA's kept pages are in its shared memory
+  // the sel rows are written while the cluster's other heads finish (nothing in
+  // the cluster reads them)
+  if (ranked) put_kept<KPT>(p, rows, take, first_pos, total);
   cluster_wait_acquire();
   if (crank != 0) {
     cluster_arrive_relaxed();  // the first CTA arrives here once it has read s_take: stay until then
