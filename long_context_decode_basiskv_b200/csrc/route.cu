@@ -390,7 +390,9 @@ __device__ __forceinline__ void put_kept(const RouteParams& p, const SelRows& ro
 // modes.  The G CTAs of a KV group run as one thread-block cluster: each keeps
 // its head's kept pages as bits in its own shared memory, and after a cluster
 // barrier the first CTA reads the others' bits (distributed shared memory),
-// forms the head mask of every page and writes the group's union list.
+// forms the head mask of every page and writes the group's union list.  Each
+// CTA writes its sel row between its cluster arrive and wait, beside the
+// cluster's other heads still ranking (nothing in the cluster reads it).
 template <int KPT>
 __global__ void __launch_bounds__(kSelectThreads) route_select_kernel(RouteParams p) {
   __shared__ int red[2 * kSelectWarps];
